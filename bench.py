@@ -1,0 +1,357 @@
+"""Benchmark of the ISA attention forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl isa|reference]
+                    [--config 480p] [--no-cpu-baseline] [--no-e2e]
+
+A step is one pass of the whole ISA forward (pre-selection, sharpness and
+routing, full attention for routed queries, Taylor attention for the rest)
+over one batch of the 480p-latent workload (B=1, H=24, d=128, 20280 source +
+20280 context tokens, block 128, keep 0.25, rho 0.2; seeded synthetic bf16
+inputs).  q, k, v (747 MB) are larger than the 126 MB L2, so no flush is
+needed between steps.  Timing: CUDA events on the launching stream around
+exactly K steps after W warm-up steps, barrier + synchronize on both sides,
+max over ranks.  With N > 1 (torchrun), every rank runs its own replica of
+the workload (heads are independent units: no collective on the data path).
+
+--impl reference times the float64 CPU oracle on the host cores instead
+(rank 0 only), one sampled head per step, scaled to a whole step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, bf16_bits_to_f64, head_inputs, make_inputs, to_torch_bf16  # noqa: E402
+
+METRIC = "ISA attn fwd latency (ms), eff. TFLOP/s vs in-house dense kernel, 1×B200"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def counts(cfg):
+    """Static per-head sizes of the ISA reading (block layout, kept / routed counts)."""
+    import math
+
+    nSB = -(-cfg.N_src // cfg.block)
+    nCB = -(-cfg.N_ctx // cfg.block)
+    n_keep = int(min(max(math.ceil(cfg.keep * nCB - 1e-6 * nCB), 0), nCB))
+    n_route = int(min(max(math.ceil(cfg.rho * cfg.N - 1e-6 * cfg.N), 0), cfg.N))
+    return nSB, nCB, n_keep, n_route
+
+
+def work_model(cfg, kept_tokens_mean):
+    """Executed FLOPs and algorithmic bytes of one step (all heads)."""
+    nSB, nCB, n_keep, n_route = counts(cfg)
+    BH, N, d = cfg.B * cfg.H, cfg.N, cfg.d
+    nK = nSB + n_keep
+    T = kept_tokens_mean
+    return dict(
+        dense_flops=4.0 * BH * N * N * d,
+        full_flops=4.0 * BH * d * n_route * T,
+        taylor_flops=4.0 * BH * d * (N - n_route) * nK,
+        sharp_flops=2.0 * 2.0 * BH * d * N * nK,
+        # algorithmic bytes of the full-attention kernel: routed Q rows and O
+        # rows once, K and V of the kept tokens once per head (L2 reuse)
+        full_bytes=BH * (2 * n_route * d * 2 + 2 * T * d * 2),
+    )
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_ms_per_step(cfg, heads, seed=0):
+    """Wall time of the float64 oracle on `heads` of the workload, scaled to a
+    whole step (all B*H heads).  Returns (ms_per_step, seconds_measured)."""
+    import oracle  # the CPU baseline leg is the one place bench.py runs the oracle
+
+    t_total = 0.0
+    for h in heads:
+        q, k, v = (bf16_bits_to_f64(x) for x in head_inputs(cfg, 0, h, seed))
+        t0 = time.perf_counter()
+        oracle.isa_head(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+        t_total += time.perf_counter() - t0
+    return 1e3 * t_total / len(heads) * cfg.B * cfg.H, t_total
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cores = len(os.sched_getaffinity(0))
+    nh = cfg.B * cfg.H
+    for s in range(args.warmup):
+        cpu_oracle_ms_per_step(cfg, [s % nh])
+    per = []
+    for s in range(args.steps):
+        ms, _ = cpu_oracle_ms_per_step(cfg, [(args.warmup + s) % nh])
+        per.append(ms)
+    v = float(np.mean(per))
+    rec = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": config_dict(cfg, args.gpus),
+           "cpu_baseline": {"value": round(v, 3), "unit": "ms", "cores": cores, "kind": "oracle",
+                            "sample": f"1 of {nh} heads per step, scaled x{nh}"},
+           "e2e": {"value": round(v, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(rec), flush=True)
+
+
+def config_dict(cfg, n):
+    return {"workload": f"ISA fwd {cfg.name}-latent: B={cfg.B} H={cfg.H} d={cfg.d} N_src={cfg.N_src} "
+                        f"N_ctx={cfg.N_ctx} block={cfg.block} keep={cfg.keep} rho={cfg.rho}",
+            "B": cfg.B, "H": cfg.H, "d": cfg.d, "N_src": cfg.N_src, "N_ctx": cfg.N_ctx, "block": cfg.block,
+            "keep": cfg.keep, "rho": cfg.rho, "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
+            "l2": "inputs (747 MB) larger than L2, no flush"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="isa", choices=["isa", "reference"])
+    ap.add_argument("--config", default="480p")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    args = ap.parse_args()
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from sparse_attention_context_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    bits = make_inputs(cfg, seed=rank)
+    q, k, v = (to_torch_bf16(b).to(dev) for b in bits)
+    shape = api.make_shape(q, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    ws = api.new_workspace(shape, dev)
+    nSB, nCB, n_keep, n_route = counts(cfg)
+    B, H, N = cfg.B, cfg.H, cfg.N
+    kept = torch.empty((B, H, n_keep), dtype=torch.int32, device=dev)
+    routed = torch.empty((B, H, n_route), dtype=torch.int32, device=dev)
+    taylor = torch.empty((B, H, N - n_route), dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    ev_full = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+
+    def step(i=None):
+        e = stage_ev[i] if i is not None else None
+        if e: e[0].record(stream)
+        api.isa_preselect_ctx(q, k, v, shape, ws, kept=kept, want_saliency=False)
+        if e: e[1].record(stream)
+        api.isa_route_queries(q, kept, shape, ws, routed=routed, taylor=taylor, want_sharpness=False)
+        if e: e[2].record(stream)
+        api.isa_full_attn_fwd(q, k, v, kept, routed, shape, ws, out)
+        if e: e[3].record(stream)
+        api.isa_taylor_attn_fwd(q, kept, taylor, shape, ws, out)
+        if e: e[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert api.isa_read_device_status(ws) == 0
+    # kept token count (for the work model), from the kept set of this input
+    kept_h = kept.cpu().numpy().reshape(B * H, n_keep)
+    tok = []
+    for row in kept_h:
+        ctx = sum(min(cfg.block, cfg.N_ctx - c * cfg.block) for c in row)
+        tok.append(cfg.N_src + ctx)
+    T_mean = float(np.mean(tok))
+    wm = work_model(cfg, T_mean)
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    stage_ms = np.array([[stage_ev[i][j].elapsed_time(stage_ev[i][j + 1]) for j in range(4)]
+                         for i in range(args.steps)]).mean(axis=0)
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    assert api.isa_read_device_status(ws) == 0
+
+    # in-house dense kernel on the same inputs (the baseline the metric names)
+    dense_ms = None
+    if not args.no_dense:
+        dws = api.dense_workspace(dev)
+        dout = torch.empty_like(q)
+        nd = max(2, min(args.steps, 5))
+        for _ in range(2):
+            api.isa_dense_attn_fwd(q, k, v, out=dout, ws=dws)
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(nd):
+            api.isa_dense_attn_fwd(q, k, v, out=dout, ws=dws)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = d0.elapsed_time(d1) / nd
+        assert api.isa_read_device_status(dws) == 0
+        del dout
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (to_torch_bf16(b).pin_memory() for b in bits)
+        hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        for _ in range(2):
+            api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws, out=hout)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ne = max(2, min(args.steps, 5))
+        e0.record(stream)
+        for _ in range(ne):
+            api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws, out=hout)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / ne
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": 3 * q.numel() * 2,
+               "d2h_bytes_per_step": q.numel() * 2}
+
+    pk, pk_kind = peaks()
+    full_ms = float(stage_ms[2])
+    ach = wm["full_flops"] / (full_ms * 1e-3) / 1e12
+    roof = {"kernel": "full_attn_routed (flash_kernel<128,128,FULL>)", "bound": "tensor",
+            "achieved": round(ach, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(ach / pk["bf16_tflops"], 4), "peak_kind": f"{pk_kind} burst bf16",
+            "frac_of_sustained": round(ach / pk["bf16_tflops_sustained"], 4),
+            "traffic": None, "kernel_ms": round(full_ms, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cms, secs = cpu_oracle_ms_per_step(cfg, [0, cfg.H - 1])
+        cpu = {"value": round(cms, 1), "unit": "ms", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"heads 0 and {cfg.H - 1} of {cfg.B * cfg.H} ({secs:.1f} s of CPU work), "
+                         f"scaled x{cfg.B * cfg.H / 2:g}"}
+
+    launches_per_step = 3 + 3 + (1 if n_route > 0 else 0) + (2 if N - n_route > 0 else 0)
+    if rank == 0:
+        rec = {"metric": METRIC, "value": round(ms_max, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": False,
+               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+               "config": config_dict(cfg, world),
+               "eff_tflops": round(wm["dense_flops"] / (ms_max * 1e-3) / 1e12, 1),
+               "dense_ms": None if dense_ms is None else round(dense_ms, 4),
+               "isa_over_dense": None if dense_ms is None else round(ms_max / dense_ms, 4),
+               "dense_tflops": None if dense_ms is None else round(wm["dense_flops"] / (dense_ms * 1e-3) / 1e12, 1),
+               "stage_ms": {"preselect": round(float(stage_ms[0]), 4), "route": round(float(stage_ms[1]), 4),
+                            "full_attn": round(float(stage_ms[2]), 4), "taylor_attn": round(float(stage_ms[3]), 4)},
+               "executed_tflop": round((wm["full_flops"] + wm["taylor_flops"] + wm["sharp_flops"]) / 1e12, 4),
+               "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+               "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
+        print(json.dumps(rec), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

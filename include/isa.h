@@ -1,0 +1,154 @@
+/*
+ * isa.h -- C ABI of the In-context Sparse Attention (ISA) forward, sm_100a.
+ *
+ * Method: "Lightning Unified Video Editing via In-Context Sparse Attention"
+ * (Shao et al., 2026), abstract.  The sequence of every (batch, head) holds
+ * N_src source-video tokens followed by N_ctx context tokens.  ISA runs in
+ * four stages, each a call (or part of a call) below:
+ *   1. context pre-selection   (abstract, first insight: context tokens are
+ *      less salient; redundant context is pruned)      -> isa_preselect_ctx
+ *   2. query sharpness + dynamic query grouping (abstract, second insight:
+ *      sharpness tracks approximation error)            -> isa_route_queries
+ *   3. full attention for the routed (sharp) queries    -> isa_attn_fwd
+ *   4. 0-th order Taylor sparse attention for the rest  -> isa_attn_fwd
+ * The abstract gives only this outline; the formulas implemented are:
+ *   blocks   per segment, `block` tokens each, the last one of each segment
+ *            partial; cnt_b tokens in block b; Xbar_b = block mean of x.
+ *   s        scale (1/sqrt(d) when shape->scale <= 0).
+ *   saliency sal_c = sum_r cnt_r * softmax_c(s Qbar_r.Kbar_c + ln cnt_c) / N
+ *            over all key blocks c; context blocks ranked by it; the top
+ *            n_keep = ceil(keep*nCB - 1e-6*nCB) are kept; source blocks always.
+ *   sharp_i  max_b softmax_b(s q_i.Kbar_b + ln cnt_b) over kept blocks.
+ *   routing  the n_route = ceil(rho*N - 1e-6*N) sharpest queries (ties: lower
+ *            index first) -> full attention over every token of every kept
+ *            block; the others -> sum_b cnt_b e^{s q.Kbar_b} Vbar_b /
+ *            sum_b cnt_b e^{s q.Kbar_b} over kept blocks.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every tensor pointer is a DEVICE pointer owned by the caller, 16-byte
+ *   aligned.  q, k, v, out are contiguous [B, H, N, d] bf16 (given here as
+ *   uint16_t bit patterns), d innermost, N = N_src + N_ctx; rows 0..N_src-1
+ *   of each head are source tokens, the rest context tokens.
+ * - Index outputs are int32, ascending within each (b, h).
+ * - The library allocates no memory and keeps no state between calls; all
+ *   scratch lives in the caller's workspace `ws` of `ws_bytes` bytes
+ *   (16-byte aligned), sized by isa_workspace_size().  The first 256 bytes
+ *   of `ws` are a control block: an int32 device status word at offset 0
+ *   (0 = no error) and an int32 fault-injection word at offset 4 (tests
+ *   only; leave it 0).  Zero the control block once after allocating ws.
+ * - Calls validate every argument before launching anything and return an
+ *   isa_status; on an error nothing is launched.  Launches are asynchronous
+ *   on `stream` (a cudaStream_t; NULL = legacy default stream).  A kernel
+ *   that gives up on a bounded wait writes ISA_ERR_DEVICE_TIMEOUT into the
+ *   status word and exits; read it with isa_read_device_status().
+ * - Supported: d in {64, 128}; block in {64, 128}; N_src >= 1; N_ctx >= 0;
+ *   0 <= keep <= 1; 0 <= rho <= 1; ceil(N_ctx/block) <= 4096;
+ *   B*H <= 65535.  Anything else returns ISA_ERR_UNSUPPORTED.
+ */
+#ifndef ISA_H_
+#define ISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ISA_OK = 0,
+  ISA_ERR_INVALID_ARG = 1,    /* null pointer, misalignment, negative size */
+  ISA_ERR_UNSUPPORTED = 2,    /* valid but outside the supported shapes */
+  ISA_ERR_WORKSPACE = 3,      /* ws_bytes smaller than required */
+  ISA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
+  ISA_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait expired */
+} isa_status;
+
+/* Problem shape.  scale <= 0 selects 1/sqrt(d). */
+typedef struct {
+  int B, H, N_src, N_ctx, d, block;
+  float keep, rho, scale;
+} isa_shape;
+
+/* Number of kept context blocks per (b, h): ceil(keep*nCB - 1e-6*nCB), nCB =
+ * ceil(N_ctx/block).  Returns -1 on an invalid shape. */
+int isa_n_keep(const isa_shape* shape);
+
+/* Number of routed queries per (b, h): ceil(rho*N - 1e-6*N).  -1 if invalid. */
+int isa_n_route(const isa_shape* shape);
+
+/* Bytes of workspace needed by every ISA call on this shape (0 if invalid). */
+size_t isa_workspace_size(const isa_shape* shape);
+
+/* Stage 1, context pre-selection.
+ * Computes the block means of q, k, v (kept in ws for the later calls), the
+ * saliency of every context block and the n_keep most salient ones.
+ *   kept_ctx_idx [B, H, n_keep] int32 out: context block numbers (0-based
+ *                within the context segment), ascending.  May be NULL only
+ *                when n_keep == 0.
+ *   saliency     [B, H, nCB] float out, or NULL.
+ * The block means written into ws are inputs of isa_route_queries and
+ * isa_attn_fwd; call this first with the same ws. */
+int isa_preselect_ctx(const isa_shape* shape, const uint16_t* q, const uint16_t* k,
+                      const uint16_t* v, int32_t* kept_ctx_idx, float* saliency,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Stage 2, query sharpness and dynamic grouping.
+ * Uses the block means in ws (from isa_preselect_ctx) and the kept set.
+ *   kept_ctx_idx [B, H, n_keep] int32 in (ascending, distinct, < nCB).
+ *   routed_idx   [B, H, n_route] int32 out: the sharpest queries, ascending.
+ *   taylor_idx   [B, H, N - n_route] int32 out: every other query, ascending.
+ *   sharpness    [B, H, N] float out, or NULL.
+ * routed_idx / taylor_idx may be NULL when their size is 0. */
+int isa_route_queries(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
+                      int32_t* routed_idx, int32_t* taylor_idx, float* sharpness,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Stages 3 and 4: full attention for routed_idx rows, 0-th order Taylor
+ * attention for taylor_idx rows; writes every row of out [B, H, N, d] bf16
+ * exactly once when routed_idx and taylor_idx partition 0..N-1.  Uses the
+ * block means in ws (from isa_preselect_ctx). */
+int isa_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                 const int32_t* kept_ctx_idx, const int32_t* routed_idx, const int32_t* taylor_idx,
+                 uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Stage 3 alone: full attention for the routed_idx rows of out over every
+ * token of every source block and of the kept context blocks (the part of
+ * isa_attn_fwd that does not need the block means).  Independent of stage 4:
+ * the two may run concurrently on different streams (disjoint rows of out). */
+int isa_full_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      const int32_t* kept_ctx_idx, const int32_t* routed_idx, uint16_t* out,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Stage 4 alone: 0-th order Taylor attention for the taylor_idx rows of out
+ * over the kept block means (block means in ws from isa_preselect_ctx). */
+int isa_taylor_attn_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
+                        const int32_t* taylor_idx, uint16_t* out, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* All four stages in order on one stream, with the kept set and the routed
+ * and Taylor index sets held inside ws.  out [B, H, N, d] bf16. */
+int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/* In-house dense flash attention (the latency baseline; equals ISA at
+ * keep = rho = 1): out = softmax(scale q k^T) v over all N keys, per (b, h),
+ * non-causal.  scale <= 0 selects 1/sqrt(d).  ws is a control block of at
+ * least isa_dense_workspace_size() bytes (status word as above). */
+size_t isa_dense_workspace_size(void);
+int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* q,
+                       const uint16_t* k, const uint16_t* v, uint16_t* out,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the device status word of ws (an
+ * isa_status) and resets it to 0.  Returns ISA_ERR_CUDA if reading fails. */
+int isa_read_device_status(void* ws, void* stream);
+
+/* Static description of a status code. */
+const char* isa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ISA_H_ */

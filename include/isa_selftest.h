@@ -1,0 +1,24 @@
+/*
+ * isa_selftest.h -- test-only export of libisa.so (not part of the ISA method).
+ *
+ * isa_selftest_umma runs ONE tile of the tensor-core building blocks used by
+ * the attention kernels, so that a wrong shared-memory or instruction
+ * descriptor shows up as a wrong product rather than as a wrong attention
+ * output.  All pointers are device pointers, row-major, 16-byte aligned:
+ *   A [128, d] bf16, B [bn, d] bf16      -> S [128, bn] fp32 = A B^T
+ *   P [128, bn] bf16, V [bn, d] bf16     -> O [128, d] fp32  = P V
+ * d and bn in {64, 128}.  ws: >= 256 bytes, zeroed; its first int32 receives
+ * ISA_ERR_DEVICE_TIMEOUT if a bounded wait expires.  Asynchronous on stream.
+ */
+#ifndef ISA_SELFTEST_H_
+#define ISA_SELFTEST_H_
+#include <stdint.h>
+#ifdef __cplusplus
+extern "C" {
+#endif
+int isa_selftest_umma(int d, int bn, const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V,
+                      float* S, float* O, void* ws, void* stream);
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -24,10 +24,10 @@ The exact formulas below are the plainest reading of that outline:
 * saliency of key block c: mean over query blocks r (weighted by cnt_r) of
   the block-level attention softmax_c( s * Qbar_r . Kbar_c + ln cnt_c ),
   over all key blocks; context blocks are ranked by it and the top
-  n_keep = ceil(keep * nCB - 1e-6) are kept, all source blocks always kept;
+  n_keep = ceil(keep*nCB - 1e-6*nCB) are kept, all source blocks always kept;
 * sharpness of query i: the largest probability of the block-level
   distribution softmax_b( s * q_i . Kbar_b + ln cnt_b ) over kept blocks;
-* routing: the n_route = ceil(rho * N - 1e-6) sharpest queries get full
+* routing: the n_route = ceil(rho*N - 1e-6*N) sharpest queries get full
   attention over every kept token; ties rank the lower index first;
 * 0-th order Taylor attention: exp(s q.k_j) is replaced by exp(s q.Kbar_b)
   for every j in block b, in numerator and denominator; summing over the
@@ -54,16 +54,18 @@ NEG_INF = -np.inf
 # ---------------------------------------------------------------------------
 
 def n_keep_of(keep: float, nCB: int) -> int:
-    """Number of context blocks kept: ceil(keep*nCB - 1e-6) clamped to [0, nCB].
+    """Number of context blocks kept: ceil(keep*nCB - 1e-6*nCB) in [0, nCB].
 
-    The 1e-6 guard keeps exact products such as 0.25*256 from rounding up.
+    The relative guard keeps exact products such as 0.25*256 from rounding up
+    when the fraction arrives as a float32 (0.25f*256 is exact, 0.2f*40560
+    is 8112.0001).
     """
-    return int(min(max(math.ceil(keep * nCB - 1e-6), 0), nCB))
+    return int(min(max(math.ceil(keep * nCB - 1e-6 * nCB), 0), nCB))
 
 
 def n_route_of(rho: float, N: int) -> int:
-    """Number of queries routed to full attention: ceil(rho*N - 1e-6) in [0, N]."""
-    return int(min(max(math.ceil(rho * N - 1e-6), 0), N))
+    """Number of queries routed to full attention: ceil(rho*N - 1e-6*N) in [0, N]."""
+    return int(min(max(math.ceil(rho * N - 1e-6 * N), 0), N))
 
 
 def block_layout(N_src: int, N_ctx: int, blk: int):

@@ -1,0 +1,184 @@
+"""Python binding of libisa.so: argument marshalling only.
+
+Every function takes torch tensors for device memory and the current torch
+CUDA stream, and calls the C entry point of the same name (include/isa.h);
+no step of the ISA path runs in Python or torch.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import IsaShape, check, lib
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _check_qkv(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("q, k, v, out must be contiguous CUDA bf16 tensors [B, H, N, d]")
+
+
+def make_shape(q: torch.Tensor, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0) -> IsaShape:
+    B, H, N, d = q.shape
+    return IsaShape(B, H, int(N_src), int(N - N_src), d, int(block), float(keep), float(rho), float(scale))
+
+
+def isa_n_keep(shape: IsaShape) -> int:
+    return lib().isa_n_keep(ctypes.byref(shape))
+
+
+def isa_n_route(shape: IsaShape) -> int:
+    return lib().isa_n_route(ctypes.byref(shape))
+
+
+def isa_workspace_size(shape: IsaShape) -> int:
+    return lib().isa_workspace_size(ctypes.byref(shape))
+
+
+def new_workspace(shape: IsaShape, device="cuda") -> torch.Tensor:
+    """Zeroed workspace (control block included) for every call on `shape`."""
+    n = isa_workspace_size(shape)
+    if n == 0:
+        raise ValueError("invalid or unsupported shape")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def isa_preselect_ctx(q, k, v, shape: IsaShape, ws, kept=None, saliency=None, want_saliency=True, stream=None):
+    """Stage 1.  Returns (kept_ctx_idx [B,H,n_keep] int32, saliency [B,H,nCB] or None)."""
+    _check_qkv(q, k, v)
+    B, H = shape.B, shape.H
+    nk = isa_n_keep(shape)
+    nCB = -(-shape.N_ctx // shape.block)
+    if kept is None:
+        kept = torch.empty((B, H, nk), dtype=torch.int32, device=q.device)
+    if saliency is None and want_saliency:
+        saliency = torch.empty((B, H, nCB), dtype=torch.float32, device=q.device)
+    rc = lib().isa_preselect_ctx(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                 _ptr(kept) if nk > 0 else None, _ptr(saliency), ws.data_ptr(), ws.numel(),
+                                 _stream(stream))
+    check("isa_preselect_ctx", rc)
+    return kept, saliency
+
+
+def isa_route_queries(q, kept, shape: IsaShape, ws, routed=None, taylor=None, sharpness=None, want_sharpness=True,
+                      stream=None):
+    """Stage 2.  Returns (routed_idx [B,H,n_route], taylor_idx [B,H,N-n_route], sharpness [B,H,N] or None)."""
+    _check_qkv(q)
+    B, H, N = shape.B, shape.H, shape.N_src + shape.N_ctx
+    nr = isa_n_route(shape)
+    if routed is None:
+        routed = torch.empty((B, H, nr), dtype=torch.int32, device=q.device)
+    if taylor is None:
+        taylor = torch.empty((B, H, N - nr), dtype=torch.int32, device=q.device)
+    if sharpness is None and want_sharpness:
+        sharpness = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = lib().isa_route_queries(ctypes.byref(shape), q.data_ptr(), _ptr(kept) if kept.numel() else None,
+                                 _ptr(routed) if nr > 0 else None, _ptr(taylor) if N - nr > 0 else None,
+                                 _ptr(sharpness), ws.data_ptr(), ws.numel(), _stream(stream))
+    check("isa_route_queries", rc)
+    return routed, taylor, sharpness
+
+
+def isa_attn_fwd(q, k, v, kept, routed, taylor, shape: IsaShape, ws, out=None, stream=None):
+    """Stages 3 and 4.  Returns out [B,H,N,d] bf16."""
+    if out is None:
+        out = torch.empty_like(q)
+    _check_qkv(q, k, v, out)
+    rc = lib().isa_attn_fwd(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                            _ptr(kept) if kept.numel() else None, _ptr(routed) if routed.numel() else None,
+                            _ptr(taylor) if taylor.numel() else None, out.data_ptr(), ws.data_ptr(), ws.numel(),
+                            _stream(stream))
+    check("isa_attn_fwd", rc)
+    return out
+
+
+def isa_full_attn_fwd(q, k, v, kept, routed, shape: IsaShape, ws, out, stream=None):
+    """Stage 3 only: full attention for the routed rows of `out`."""
+    _check_qkv(q, k, v, out)
+    rc = lib().isa_full_attn_fwd(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                 _ptr(kept) if kept.numel() else None, _ptr(routed) if routed.numel() else None,
+                                 out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+    check("isa_full_attn_fwd", rc)
+    return out
+
+
+def isa_taylor_attn_fwd(q, kept, taylor, shape: IsaShape, ws, out, stream=None):
+    """Stage 4 only: 0-th order Taylor attention for the taylor rows of `out`."""
+    _check_qkv(q, out)
+    rc = lib().isa_taylor_attn_fwd(ctypes.byref(shape), q.data_ptr(), _ptr(kept) if kept.numel() else None,
+                                   _ptr(taylor) if taylor.numel() else None, out.data_ptr(), ws.data_ptr(),
+                                   ws.numel(), _stream(stream))
+    check("isa_taylor_attn_fwd", rc)
+    return out
+
+
+def isa_forward(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, ws=None, out=None,
+                stream=None):
+    """All ISA stages in one call.
+
+    CUDA inputs: runs on the current stream and returns a CUDA tensor.
+    CPU inputs (the host-buffer path): copies q, k, v to the GPU, runs, and
+    copies the output back into a pinned CPU tensor (returned).
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda")
+        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    shape = make_shape(q, N_src, block, keep, rho, scale)
+    if ws is None:
+        ws = new_workspace(shape, q.device)
+    o = torch.empty_like(q) if (out is None or host) else out
+    _check_qkv(q, k, v, o)
+    rc = lib().isa_forward(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                           ws.data_ptr(), ws.numel(), _stream(stream))
+    check("isa_forward", rc)
+    if host:
+        dst = out if out is not None else torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        dst.copy_(o, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return dst
+    return o
+
+
+def dense_workspace(device="cuda") -> torch.Tensor:
+    return torch.zeros(lib().isa_dense_workspace_size(), dtype=torch.uint8, device=device)
+
+
+def isa_dense_attn_fwd(q, k, v, scale: float = 0.0, out=None, ws=None, stream=None):
+    """In-house dense flash attention (the baseline).  Returns out [B,H,N,d] bf16."""
+    if out is None:
+        out = torch.empty_like(q)
+    _check_qkv(q, k, v, out)
+    if ws is None:
+        ws = dense_workspace(q.device)
+    B, H, N, d = q.shape
+    rc = lib().isa_dense_attn_fwd(B, H, N, d, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                  out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+    check("isa_dense_attn_fwd", rc)
+    return out
+
+
+def isa_read_device_status(ws, stream=None) -> int:
+    """Synchronise, return the device status word of `ws` and reset it."""
+    return lib().isa_read_device_status(ws.data_ptr(), _stream(stream))
+
+
+def isa_selftest_umma(A, B, P, V, ws, stream=None):
+    """Test-only: one-tile UMMA products S = A B^T and O = P V (fp32)."""
+    d, bn = A.shape[1], B.shape[0]
+    S = torch.empty((128, bn), dtype=torch.float32, device=A.device)
+    O = torch.empty((128, d), dtype=torch.float32, device=A.device)
+    rc = lib().isa_selftest_umma(d, bn, A.data_ptr(), B.data_ptr(), P.data_ptr(), V.data_ptr(), S.data_ptr(),
+                                 O.data_ptr(), ws.data_ptr(), _stream(stream))
+    check("isa_selftest_umma", rc)
+    return S, O

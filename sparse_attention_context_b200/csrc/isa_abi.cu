@@ -1,0 +1,440 @@
+// isa_abi.cu -- the C ABI declared in include/isa.h: argument validation,
+// workspace layout, tensor-map encoding and the launch sequence of every
+// ISA stage.  Host code only; the arithmetic lives in the kernel files.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "isa.h"
+#include "isa_internal.h"
+
+namespace isa {
+namespace {
+
+struct Dims {
+  int B, H, BH, N_src, N_ctx, N, d, blk, nSB, nCB, nB, n_keep, n_route, nK, nKpad, nChunks;
+  float scale;
+};
+
+struct WsLayout {
+  size_t Qbar, Kbar, Vbar, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int keep_count(float keep, int nCB) {
+  const double v = std::ceil(static_cast<double>(keep) * nCB - 1e-6 * nCB);
+  return static_cast<int>(std::min<double>(std::max<double>(v, 0.0), nCB));
+}
+int route_count(float rho, int N) {
+  const double v = std::ceil(static_cast<double>(rho) * N - 1e-6 * N);
+  return static_cast<int>(std::min<double>(std::max<double>(v, 0.0), N));
+}
+
+int check_shape(const isa_shape* s, Dims* o) {
+  if (s == nullptr) return ISA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->H < 1 || s->N_src < 1 || s->N_ctx < 0) return ISA_ERR_INVALID_ARG;
+  if (!(s->keep >= 0.f && s->keep <= 1.f) || !(s->rho >= 0.f && s->rho <= 1.f)) return ISA_ERR_INVALID_ARG;
+  if (!std::isfinite(s->scale)) return ISA_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return ISA_ERR_UNSUPPORTED;
+  if (s->block != 64 && s->block != 128) return ISA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(s->B) * s->H;
+  const long long N = static_cast<long long>(s->N_src) + s->N_ctx;
+  if (BH > 65535) return ISA_ERR_UNSUPPORTED;
+  if (BH * (N + 4096) >= INT_MAX) return ISA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  Dims d{};
+  d.B = s->B;
+  d.H = s->H;
+  d.BH = static_cast<int>(BH);
+  d.N_src = s->N_src;
+  d.N_ctx = s->N_ctx;
+  d.N = static_cast<int>(N);
+  d.d = s->d;
+  d.blk = s->block;
+  d.nSB = (d.N_src + d.blk - 1) / d.blk;
+  d.nCB = (d.N_ctx + d.blk - 1) / d.blk;
+  if (d.nCB > kTopkCap) return ISA_ERR_UNSUPPORTED;
+  d.nB = d.nSB + d.nCB;
+  d.n_keep = keep_count(s->keep, d.nCB);
+  d.n_route = route_count(s->rho, d.N);
+  d.nK = d.nSB + d.n_keep;
+  d.nKpad = (d.nK + 127) / 128 * 128;
+  d.nChunks = (d.nB + kSalRows - 1) / kSalRows;
+  d.scale = s->scale > 0.f ? s->scale : 1.0f / std::sqrt(static_cast<float>(d.d));
+  *o = d;
+  return ISA_OK;
+}
+
+WsLayout layout(const Dims& d) {
+  WsLayout L{};
+  size_t off = kCtlBytes;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  const size_t BH = d.BH;
+  L.Qbar = take(BH * d.nB * d.d * 4);
+  L.Kbar = take(BH * d.nB * d.d * 4);
+  L.Vbar = take(BH * d.nB * d.d * 4);
+  L.partial = take(BH * d.nChunks * std::max(d.nCB, 1) * 4);
+  L.sal = take(BH * std::max(d.nCB, 1) * 4);
+  L.Khi = take(BH * d.nKpad * d.d * 2);
+  L.Klo = take(BH * d.nKpad * d.d * 2);
+  L.Vb = take(BH * d.nKpad * d.d * 2);
+  L.bias2 = take(BH * d.nKpad * 4);
+  L.sharp = take(BH * d.N * 4);
+  L.kept = take(BH * std::max(d.n_keep, 1) * 4);
+  L.routed = take(BH * std::max(d.n_route, 1) * 4);
+  L.taylor = take(BH * std::max(d.N - d.n_route, 1) * 4);
+  L.total = off;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || !aligned16(ws)) return ISA_ERR_INVALID_ARG;
+  if (ws_bytes < need) return ISA_ERR_WORKSPACE;
+  return ISA_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? ISA_OK : ISA_ERR_CUDA; }
+
+// --- tensor maps (driver entry point fetched once through the runtime)
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Common pieces of the stage launches.
+struct Ctx {
+  Dims d;
+  WsLayout L;
+  void* ws;
+  cudaStream_t st;
+  int* status() const { return at<int>(ws, kStatusOffset); }
+  const int* inject() const { return at<int>(ws, kInjectOffset); }
+};
+
+FlashParams base_params(const Ctx& c) {
+  FlashParams p{};
+  p.N = c.d.N;
+  p.N_src = c.d.N_src;
+  p.N_ctx = c.d.N_ctx;
+  p.blk = c.d.blk;
+  p.nSB = c.d.nSB;
+  p.n_keep = c.d.n_keep;
+  p.scale_log2 = c.d.scale * 1.4426950408889634f;
+  p.status = c.status();
+  p.inject = c.inject();
+  return p;
+}
+
+int run_preselect(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, int32_t* kept,
+                  float* sal_user) {
+  const Dims& d = c.d;
+  cudaError_t e = launch_pool(q, k, v, at<float>(c.ws, c.L.Qbar), at<float>(c.ws, c.L.Kbar),
+                              at<float>(c.ws, c.L.Vbar), d.BH, d.N_src, d.N_ctx, d.d, d.blk, c.st);
+  if (e == cudaSuccess)
+    e = launch_saliency(at<float>(c.ws, c.L.Qbar), at<float>(c.ws, c.L.Kbar), at<float>(c.ws, c.L.partial), d.BH,
+                        d.N_src, d.N_ctx, d.d, d.blk, d.scale, c.st);
+  if (e == cudaSuccess)
+    e = launch_select_ctx(at<float>(c.ws, c.L.partial), at<float>(c.ws, c.L.sal), sal_user, kept, d.BH, d.N_src,
+                          d.N_ctx, d.blk, d.n_keep, c.st);
+  return cuda_status(e);
+}
+
+int run_build_kept(const Ctx& c, const int32_t* kept) {
+  const Dims& d = c.d;
+  return cuda_status(launch_build_kept(at<float>(c.ws, c.L.Kbar), at<float>(c.ws, c.L.Vbar), kept,
+                                       at<uint16_t>(c.ws, c.L.Khi), at<uint16_t>(c.ws, c.L.Klo),
+                                       at<uint16_t>(c.ws, c.L.Vb), at<float>(c.ws, c.L.bias2), d.BH, d.N_src,
+                                       d.N_ctx, d.d, d.blk, d.n_keep, d.nKpad, c.status(), c.st));
+}
+
+int run_route(const Ctx& c, const uint16_t* q, const int32_t* kept, int32_t* routed, int32_t* taylor,
+              float* sharp_user) {
+  const Dims& d = c.d;
+  int rc = run_build_kept(c, kept);
+  if (rc != ISA_OK) return rc;
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return ISA_ERR_CUDA;
+  CUtensorMap tmHi, tmLo;
+  if (!make_tmap_bf16(&tmHi, at<uint16_t>(c.ws, c.L.Khi), static_cast<uint64_t>(d.BH) * d.nKpad, d.d, 128) ||
+      !make_tmap_bf16(&tmLo, at<uint16_t>(c.ws, c.L.Klo), static_cast<uint64_t>(d.BH) * d.nKpad, d.d, 128))
+    return ISA_ERR_CUDA;
+  float* sharp = sharp_user ? sharp_user : at<float>(c.ws, c.L.sharp);
+  FlashParams p = base_params(c);
+  p.q = q;
+  p.sharp = sharp;
+  p.row_idx = nullptr;
+  p.n_rows = d.N;
+  p.n_kv_tiles = d.nKpad / 128;
+  p.kv_rows_per_head = d.nKpad;
+  p.bias2 = at<float>(c.ws, c.L.bias2);
+  cudaError_t e = launch_flash(d.d, 128, MODE_SHARP, tmHi, tmLo, p, d.BH, c.st);
+  if (e == cudaSuccess) e = launch_route(sharp, routed, taylor, d.BH, d.N, d.n_route, c.status(), c.st);
+  return cuda_status(e);
+}
+
+int run_full(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kept,
+             const int32_t* routed, uint16_t* out) {
+  const Dims& d = c.d;
+  cudaError_t e = cudaSuccess;
+  if (d.n_route > 0) {
+    CUtensorMap tmK, tmV;
+    if (!make_tmap_bf16(&tmK, k, static_cast<uint64_t>(d.BH) * d.N, d.d, d.blk) ||
+        !make_tmap_bf16(&tmV, v, static_cast<uint64_t>(d.BH) * d.N, d.d, d.blk))
+      return ISA_ERR_CUDA;
+    FlashParams p = base_params(c);
+    p.q = q;
+    p.out = out;
+    p.row_idx = routed;
+    p.n_rows = d.n_route;
+    p.kept_ctx = kept;
+    p.n_kv_tiles = d.nSB + d.n_keep;
+    p.kv_rows_per_head = d.N;
+    e = launch_flash(d.d, d.blk, MODE_FULL, tmK, tmV, p, d.BH, c.st);
+  }
+  return cuda_status(e);
+}
+
+int run_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, const int32_t* taylor, uint16_t* out,
+               bool rebuild_kept) {
+  const Dims& d = c.d;
+  if (d.N - d.n_route <= 0) return ISA_OK;
+  if (rebuild_kept) {
+    const int rc = run_build_kept(c, kept);
+    if (rc != ISA_OK) return rc;
+  }
+  cudaError_t e = cudaSuccess;
+  {
+    CUtensorMap tmK, tmV;
+    if (!make_tmap_bf16(&tmK, at<uint16_t>(c.ws, c.L.Khi), static_cast<uint64_t>(d.BH) * d.nKpad, d.d, 128) ||
+        !make_tmap_bf16(&tmV, at<uint16_t>(c.ws, c.L.Vb), static_cast<uint64_t>(d.BH) * d.nKpad, d.d, 128))
+      return ISA_ERR_CUDA;
+    FlashParams p = base_params(c);
+    p.q = q;
+    p.out = out;
+    p.row_idx = taylor;
+    p.n_rows = d.N - d.n_route;
+    p.n_kv_tiles = d.nKpad / 128;
+    p.kv_rows_per_head = d.nKpad;
+    p.bias2 = at<float>(c.ws, c.L.bias2);
+    e = launch_flash(d.d, 128, MODE_TAYLOR, tmK, tmV, p, d.BH, c.st);
+  }
+  return cuda_status(e);
+}
+
+int run_attn(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kept,
+             const int32_t* routed, const int32_t* taylor, uint16_t* out, bool rebuild_kept) {
+  int rc = run_full(c, q, k, v, kept, routed, out);
+  if (rc == ISA_OK) rc = run_taylor(c, q, kept, taylor, out, rebuild_kept);
+  return rc;
+}
+
+int make_ctx(const isa_shape* shape, void* ws, size_t ws_bytes, void* stream, Ctx* c) {
+  int rc = check_shape(shape, &c->d);
+  if (rc != ISA_OK) return rc;
+  c->L = layout(c->d);
+  rc = check_ws(ws, ws_bytes, c->L.total);
+  if (rc != ISA_OK) return rc;
+  c->ws = ws;
+  c->st = static_cast<cudaStream_t>(stream);
+  return ISA_OK;
+}
+
+bool tensors_ok(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p == nullptr || !aligned16(p)) return false;
+  return true;
+}
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace isa
+
+using namespace isa;
+
+extern "C" {
+
+int isa_n_keep(const isa_shape* shape) {
+  Dims d;
+  return check_shape(shape, &d) == ISA_OK ? d.n_keep : -1;
+}
+
+int isa_n_route(const isa_shape* shape) {
+  Dims d;
+  return check_shape(shape, &d) == ISA_OK ? d.n_route : -1;
+}
+
+size_t isa_workspace_size(const isa_shape* shape) {
+  Dims d;
+  if (check_shape(shape, &d) != ISA_OK) return 0;
+  return layout(d).total;
+}
+
+int isa_preselect_ctx(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      int32_t* kept_ctx_idx, float* saliency, void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q, k, v})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (saliency != nullptr && !aligned16(saliency)) return ISA_ERR_INVALID_ARG;
+  return run_preselect(c, q, k, v, kept_ctx_idx, saliency);
+}
+
+int isa_route_queries(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx, int32_t* routed_idx,
+                      int32_t* taylor_idx, float* sharpness, void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_route > 0 && (routed_idx == nullptr || !aligned16(routed_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.N - c.d.n_route > 0 && (taylor_idx == nullptr || !aligned16(taylor_idx))) return ISA_ERR_INVALID_ARG;
+  if (sharpness != nullptr && !aligned16(sharpness)) return ISA_ERR_INVALID_ARG;
+  return run_route(c, q, kept_ctx_idx, routed_idx, taylor_idx, sharpness);
+}
+
+int isa_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                 const int32_t* kept_ctx_idx, const int32_t* routed_idx, const int32_t* taylor_idx, uint16_t* out,
+                 void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_route > 0 && (routed_idx == nullptr || !aligned16(routed_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.N - c.d.n_route > 0 && (taylor_idx == nullptr || !aligned16(taylor_idx))) return ISA_ERR_INVALID_ARG;
+  return run_attn(c, q, k, v, kept_ctx_idx, routed_idx, taylor_idx, out, true);
+}
+
+int isa_full_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      const int32_t* kept_ctx_idx, const int32_t* routed_idx, uint16_t* out, void* ws,
+                      size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_route > 0 && (routed_idx == nullptr || !aligned16(routed_idx))) return ISA_ERR_INVALID_ARG;
+  return run_full(c, q, k, v, kept_ctx_idx, routed_idx, out);
+}
+
+int isa_taylor_attn_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
+                        const int32_t* taylor_idx, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q, out})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.N - c.d.n_route > 0 && (taylor_idx == nullptr || !aligned16(taylor_idx))) return ISA_ERR_INVALID_ARG;
+  return run_taylor(c, q, kept_ctx_idx, taylor_idx, out, true);
+}
+
+int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
+  int32_t* kept = at<int32_t>(ws, c.L.kept);
+  int32_t* routed = at<int32_t>(ws, c.L.routed);
+  int32_t* taylor = at<int32_t>(ws, c.L.taylor);
+  rc = run_preselect(c, q, k, v, kept, nullptr);
+  if (rc == ISA_OK) rc = run_route(c, q, kept, routed, taylor, nullptr);
+  if (rc == ISA_OK) rc = run_attn(c, q, k, v, kept, routed, taylor, out, false);
+  return rc;
+}
+
+size_t isa_dense_workspace_size(void) { return kCtlBytes; }
+
+int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* q, const uint16_t* k,
+                       const uint16_t* v, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  if (B < 1 || H < 1 || N < 1 || !std::isfinite(scale)) return ISA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ISA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 65535 || BH * (static_cast<long long>(N) + 128) >= INT_MAX) return ISA_ERR_UNSUPPORTED;
+  if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
+  int rc = check_ws(ws, ws_bytes, kCtlBytes);
+  if (rc != ISA_OK) return rc;
+  CUtensorMap tmK, tmV;
+  if (!make_tmap_bf16(&tmK, k, static_cast<uint64_t>(BH) * N, d, 128) ||
+      !make_tmap_bf16(&tmV, v, static_cast<uint64_t>(BH) * N, d, 128))
+    return ISA_ERR_CUDA;
+  FlashParams p{};
+  p.q = q;
+  p.out = out;
+  p.row_idx = nullptr;
+  p.n_rows = N;
+  p.N = N;
+  p.n_kv_tiles = (N + 127) / 128;
+  p.kv_rows_per_head = N;
+  p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d))) * 1.4426950408889634f;
+  p.status = at<int>(ws, kStatusOffset);
+  p.inject = at<int>(ws, kInjectOffset);
+  return cuda_status(launch_flash(d, 128, MODE_DENSE, tmK, tmV, p, static_cast<int>(BH),
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+int isa_read_device_status(void* ws, void* stream) {
+  if (ws == nullptr) return ISA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ISA_ERR_CUDA;
+  if (cudaMemcpyAsync(&h, at<int>(ws, kStatusOffset), sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return ISA_ERR_CUDA;
+  if (cudaMemsetAsync(at<int>(ws, kStatusOffset), 0, sizeof(int), st) != cudaSuccess) return ISA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ISA_ERR_CUDA;
+  return h;
+}
+
+const char* isa_status_string(int status) {
+  switch (status) {
+    case ISA_OK: return "ok";
+    case ISA_ERR_INVALID_ARG: return "invalid argument";
+    case ISA_ERR_UNSUPPORTED: return "unsupported shape";
+    case ISA_ERR_WORKSPACE: return "workspace too small";
+    case ISA_ERR_CUDA: return "CUDA error";
+    case ISA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// isa_internal.h -- launch interfaces shared by the kernel files and the
+// host ABI (isa_abi.cu).  Not part of the public C ABI.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace isa {
+
+constexpr int kStatusOffset = 0;   // int32 in the workspace control block
+constexpr int kInjectOffset = 4;   // int32 fault-injection word (tests)
+constexpr int kCtlBytes = 256;
+constexpr int kTopkCap = 4096;     // max context blocks the top-k sort holds
+constexpr int kSalRows = 16;       // query blocks per saliency CTA
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
+
+enum FlashMode { MODE_DENSE = 0, MODE_FULL = 1, MODE_TAYLOR = 2, MODE_SHARP = 3 };
+
+// Arguments of the tcgen05 attention engine (one CTA = 128 query rows of
+// one (b, h); grid = (ceil(n_rows/128), B*H)).
+struct FlashParams {
+  const uint16_t* q;      // [BH, N, D] bf16
+  uint16_t* out;          // [BH, N, D] bf16 (DENSE / FULL / TAYLOR)
+  float* sharp;           // [BH, N] fp32 (SHARP)
+  const int* row_idx;     // [BH, n_rows] gathered query rows, or null (contiguous)
+  int n_rows;             // query rows per head handled by this launch
+  int N;                  // tokens per head
+  int N_src, N_ctx, blk;  // FULL: segment sizes and block size (== BN)
+  int nSB;                // FULL: number of source blocks
+  const int* kept_ctx;    // FULL: [BH, n_keep] kept context blocks
+  int n_keep;
+  int n_kv_tiles;         // key tiles per head
+  int kv_rows_per_head;   // rows of the K/V tensor maps per head
+  const float* bias2;     // TAYLOR / SHARP: [BH, kv_rows_per_head] log2 cnt (-inf pad)
+  float scale_log2;       // s * log2(e)
+  int* status;            // device status word or null
+  const int* inject;      // device fault-injection word or null
+};
+
+// Tensor map over a [rows, D] bf16 row-major matrix, box = 64 columns x
+// box_rows rows, 128-byte swizzle.  Returns false if encoding fails.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows);
+
+cudaError_t launch_flash(int D, int BN, int mode, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                         const FlashParams& p, int BH, cudaStream_t st);
+
+// Stage-1 kernels.
+cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,
+                        float* Vbar, int BH, int N_src, int N_ctx, int D, int blk, cudaStream_t st);
+cudaError_t launch_saliency(const float* Qbar, const float* Kbar, float* partial, int BH, int N_src, int N_ctx,
+                            int D, int blk, float scale, cudaStream_t st);
+cudaError_t launch_select_ctx(const float* partial, float* sal_ws, float* sal_user, int32_t* kept, int BH,
+                              int N_src, int N_ctx, int blk, int n_keep, cudaStream_t st);
+cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_t* kept, uint16_t* Khi,
+                              uint16_t* Klo, uint16_t* Vb, float* bias2, int BH, int N_src, int N_ctx, int D,
+                              int blk, int n_keep, int nKpad, int* status, cudaStream_t st);
+cudaError_t launch_route(const float* sharp, int32_t* routed, int32_t* taylor, int BH, int N, int n_route,
+                         int* status, cudaStream_t st);
+
+}  // namespace isa

@@ -1,0 +1,80 @@
+// pool.cu -- block means of q, k, v (ISA stage 1 input; also the keys and
+// values of the 0-th order Taylor path).
+//
+// Blocks are taken per segment: source blocks b < nSB cover rows
+// [b*blk, min((b+1)*blk, N_src)), context blocks cover the context rows the
+// same way; the last block of each segment may be partial.  One CTA reduces
+// one block of one (b, h) for all three tensors: 16-byte vector loads (8
+// bf16), fp32 accumulation in a fixed order, a two-level reduction (lane
+// halves by shuffle, row groups through shared memory).  HBM-bound: every
+// byte of q, k, v is read once.
+#include "isa_internal.h"
+#include "tc_ptx.cuh"
+
+namespace isa {
+
+__device__ __forceinline__ void acc_bf16x8(float (&a)[8], const uint4& w) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    a[2 * i + 0] += __uint_as_float(u[i] << 16);
+    a[2 * i + 1] += __uint_as_float(u[i] & 0xFFFF0000u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                                                   const uint16_t* __restrict__ v, float* __restrict__ Qbar,
+                                                   float* __restrict__ Kbar, float* __restrict__ Vbar, int N_src,
+                                                   int N_ctx, int blk, int nSB, int nB) {
+  constexpr int CPR = D / 8;          // 16-byte chunks per row
+  constexpr int RG = 256 / CPR;       // row groups (rows in flight per pass)
+  __shared__ float red[3][RG][D + 4];
+  const int b = blockIdx.x, bh = blockIdx.y;
+  const int N = N_src + N_ctx;
+  const int start = b < nSB ? b * blk : N_src + (b - nSB) * blk;
+  const int cnt = b < nSB ? min(blk, N_src - b * blk) : min(blk, N_ctx - (b - nSB) * blk);
+  const int ch = threadIdx.x % CPR, rg = threadIdx.x / CPR;
+  const size_t base = (static_cast<size_t>(bh) * N + start) * D + ch * 8;
+  float aq[8] = {0}, ak[8] = {0}, av[8] = {0};
+#pragma unroll 4
+  for (int r = rg; r < cnt; r += RG) {
+    const size_t off = base + static_cast<size_t>(r) * D;
+    const uint4 wq = __ldg(reinterpret_cast<const uint4*>(q + off));
+    const uint4 wk = __ldg(reinterpret_cast<const uint4*>(k + off));
+    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(v + off));
+    acc_bf16x8(aq, wq);
+    acc_bf16x8(ak, wk);
+    acc_bf16x8(av, wv);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    red[0][rg][ch * 8 + i] = aq[i];
+    red[1][rg][ch * 8 + i] = ak[i];
+    red[2][rg][ch * 8 + i] = av[i];
+  }
+  __syncthreads();
+  const float fcnt = static_cast<float>(cnt);
+  for (int e = threadIdx.x; e < 3 * D; e += 256) {
+    const int t = e / D, col = e % D;
+    float s = 0.f;
+#pragma unroll
+    for (int g = 0; g < RG; ++g) s += red[t][g][col];
+    float* dst = t == 0 ? Qbar : (t == 1 ? Kbar : Vbar);
+    dst[(static_cast<size_t>(bh) * nB + b) * D + col] = s / fcnt;
+  }
+}
+
+cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,
+                        float* Vbar, int BH, int N_src, int N_ctx, int D, int blk, cudaStream_t st) {
+  const int nSB = (N_src + blk - 1) / blk, nCB = (N_ctx + blk - 1) / blk;
+  const int nB = nSB + nCB;
+  const dim3 grid(nB, BH);
+  if (D == 128)
+    pool_kernel<128><<<grid, 256, 0, st>>>(q, k, v, Qbar, Kbar, Vbar, N_src, N_ctx, blk, nSB, nB);
+  else
+    pool_kernel<64><<<grid, 256, 0, st>>>(q, k, v, Qbar, Kbar, Vbar, N_src, N_ctx, blk, nSB, nB);
+  return cudaGetLastError();
+}
+
+}  // namespace isa

@@ -1,0 +1,129 @@
+// selftest.cu -- a one-tile check of the UMMA building blocks used by the
+// attention engine: S = A B^T with both operands K-major (A written by
+// threads into the 128B-swizzled layout, B loaded by TMA) and O = P V with
+// V MN-major (loaded by TMA), both accumulated in TMEM and read back with
+// tcgen05.ld.  Exported for the tests only (include/isa_selftest.h).
+#include "isa.h"
+#include "isa_internal.h"
+#include "isa_selftest.h"
+#include "tc_ptx.cuh"
+
+namespace isa {
+
+template <int D, int BN>
+__global__ void __launch_bounds__(128, 1)
+    umma_probe_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmV,
+                      const uint16_t* A, const uint16_t* P, float* S_out, float* O_out, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  constexpr int A_BYTES = 128 * D * 2, B_BYTES = BN * D * 2, P_BYTES = 128 * BN * 2;
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + A_BYTES;
+  uint8_t* sV = sB + B_BYTES;
+  uint8_t* sP = sV + B_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + P_BYTES);  // [0] tma, [1] mma
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  constexpr int TMEM_COLS = (BN + D) <= 256 ? 256 : 512;
+  const int tid = threadIdx.x, warp = tid >> 5;
+
+  // A (128 x D) and P (128 x BN), K-major, written by threads.
+  for (int c = tid; c < 128 * (D / 8); c += 128) {
+    const int row = c / (D / 8), ch = c % (D / 8);
+    const uint4 val = *reinterpret_cast<const uint4*>(A + row * D + ch * 8);
+    st_shared_v4(smem_u32(sA) + (ch >> 3) * (128 * 128) + sw128(row, ch & 7), val.x, val.y, val.z, val.w);
+  }
+  for (int c = tid; c < 128 * (BN / 8); c += 128) {
+    const int row = c / (BN / 8), ch = c % (BN / 8);
+    const uint4 val = *reinterpret_cast<const uint4*>(P + row * BN + ch * 8);
+    st_shared_v4(smem_u32(sP) + (ch >> 3) * (128 * 128) + sw128(row, ch & 7), val.x, val.y, val.z, val.w);
+  }
+  fence_proxy_async_smem();
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], 2 * B_BYTES);
+    for (int c = 0; c < D / 64; ++c) tma_load_2d(sB + c * (BN * 128), &tmB, &bars[0], c * 64, 0);
+    for (int c = 0; c < D / 64; ++c) tma_load_2d(sV + c * (BN * 128), &tmV, &bars[0], c * 64, 0);
+    ok = mbar_wait_bounded(&bars[0], 0, nullptr, kWaitLimitNs) == 0;
+    if (ok) {
+      tc_fence_after();
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_bf16(tmem, desc_k_sw128(smem_u32(sA) + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                  desc_k_sw128(smem_u32(sB) + (kk >> 2) * (BN * 128) + (kk & 3) * 32), idesc_bf16(128, BN, 0),
+                  kk > 0);
+      for (int kk = 0; kk < BN / 16; ++kk)
+        umma_bf16(tmem + BN, desc_k_sw128(smem_u32(sP) + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                  desc_mn_sw128(smem_u32(sV) + kk * 16 * 128, BN * 128), idesc_bf16(128, D, 1), kk > 0);
+    }
+    umma_commit(&bars[1]);
+    if (!ok) atomicCAS(status, 0, ISA_ERR_DEVICE_TIMEOUT);
+  }
+  __syncwarp();
+  const bool done = mbar_wait_bounded(&bars[1], 0, nullptr, kWaitLimitNs) == 0;
+  ok = __all_sync(0xffffffffu, done);
+  tc_fence_after();
+  const int row = tid;
+  const uint32_t lb = static_cast<uint32_t>(warp * 32) << 16;
+  if (ok) {
+    for (int j = 0; j < BN / 32; ++j) {
+      uint32_t u[32];
+      tmem_ld32(tmem + lb + j * 32, u);
+      tmem_wait_ld();
+      for (int i = 0; i < 32; ++i) S_out[row * BN + j * 32 + i] = __uint_as_float(u[i]);
+    }
+    for (int j = 0; j < D / 32; ++j) {
+      uint32_t u[32];
+      tmem_ld32(tmem + lb + BN + j * 32, u);
+      tmem_wait_ld();
+      for (int i = 0; i < 32; ++i) O_out[row * D + j * 32 + i] = __uint_as_float(u[i]);
+    }
+  } else if (tid == 0) {
+    atomicCAS(status, 0, ISA_ERR_DEVICE_TIMEOUT);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <int D, int BN>
+static int run_probe(const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V, float* S, float* O,
+                     int* status, cudaStream_t st) {
+  CUtensorMap tmB, tmV;
+  if (!make_tmap_bf16(&tmB, B, BN, D, BN) || !make_tmap_bf16(&tmV, V, BN, D, BN)) return ISA_ERR_CUDA;
+  const int smem = 128 * D * 2 + 2 * BN * D * 2 + 128 * BN * 2 + 64 + 1024;
+  auto kern = umma_probe_kernel<D, BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ISA_ERR_CUDA;
+  kern<<<1, 128, smem, st>>>(tmB, tmV, A, P, S, O, status);
+  return cudaGetLastError() == cudaSuccess ? ISA_OK : ISA_ERR_CUDA;
+}
+
+}  // namespace isa
+
+extern "C" int isa_selftest_umma(int d, int bn, const uint16_t* A, const uint16_t* B, const uint16_t* P,
+                                 const uint16_t* V, float* S, float* O, void* ws, void* stream) {
+  if (!A || !B || !P || !V || !S || !O || !ws) return ISA_ERR_INVALID_ARG;
+  int* status = reinterpret_cast<int*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128 && bn == 128) return isa::run_probe<128, 128>(A, B, P, V, S, O, status, st);
+  if (d == 128 && bn == 64) return isa::run_probe<128, 64>(A, B, P, V, S, O, status, st);
+  if (d == 64 && bn == 128) return isa::run_probe<64, 128>(A, B, P, V, S, O, status, st);
+  if (d == 64 && bn == 64) return isa::run_probe<64, 64>(A, B, P, V, S, O, status, st);
+  return ISA_ERR_UNSUPPORTED;
+}

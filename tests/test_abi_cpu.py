@@ -1,0 +1,102 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/*.h declares, and its host-side logic (counts, workspace sizing,
+argument validation before any launch) behaves as documented."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import oracle
+from sparse_attention_context_b200 import _lib
+from sparse_attention_context_b200._lib import IsaShape
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names.update(re.findall(r"\b(isa_\w+)\s*\(", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(_lib.LIB_PATH):
+        from sparse_attention_context_b200 import build
+
+        build.build()
+    return _lib.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = declared_functions()
+    assert "isa_attn_fwd" in names and "isa_dense_attn_fwd" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_lib.SIGNATURES), "binding signatures and header disagree"
+
+
+def shape(**kw):
+    base = dict(B=1, H=24, N_src=20280, N_ctx=20280, d=128, block=128, keep=0.25, rho=0.2, scale=0.0)
+    base.update(kw)
+    return IsaShape(**base)
+
+
+@pytest.mark.parametrize("keep,rho,N_src,N_ctx,blk", [
+    (0.25, 0.2, 20280, 20280, 128), (0.5, 0.25, 256, 256, 64), (0.3, 0.2, 4096, 4096, 128),
+    (0.2, 0.15, 75600, 75600, 128), (0.0, 0.0, 100, 0, 64), (1.0, 1.0, 77, 300, 64), (0.1, 0.5, 32768, 32768, 128)])
+def test_counts_match_oracle(L, keep, rho, N_src, N_ctx, blk):
+    s = shape(N_src=N_src, N_ctx=N_ctx, block=blk, keep=keep, rho=rho)
+    nCB = -(-N_ctx // blk)
+    assert L.isa_n_keep(ctypes.byref(s)) == oracle.n_keep_of(keep, nCB)
+    assert L.isa_n_route(ctypes.byref(s)) == oracle.n_route_of(rho, N_src + N_ctx)
+
+
+def test_workspace_size(L):
+    s = shape()
+    n = L.isa_workspace_size(ctypes.byref(s))
+    # block means (3 x fp32) + gathered bf16 operands + sharpness + index sets
+    BH, N, nB, d = 24, 40560, 318, 128
+    assert n >= 3 * BH * nB * d * 4 + BH * N * 4 + BH * N * 4
+    assert n < 64 * 2**20
+    assert L.isa_workspace_size(ctypes.byref(shape(d=96))) == 0
+    assert L.isa_dense_workspace_size() >= 8
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(d=96), 2), (dict(block=32), 2), (dict(keep=1.5), 1), (dict(rho=-0.1), 1), (dict(N_src=0), 1),
+    (dict(B=0), 1), (dict(N_ctx=-1), 1), (dict(H=70000), 2), (dict(N_ctx=4097 * 64, block=64), 2)])
+def test_invalid_shapes_rejected_before_launch(L, bad, code):
+    s = shape(**bad)
+    buf = (ctypes.c_uint8 * 1024)()
+    p = ctypes.addressof(buf)
+    assert L.isa_preselect_ctx(ctypes.byref(s), p, p, p, p, None, p, 1024, None) == code
+    assert L.isa_forward(ctypes.byref(s), p, p, p, p, p, 1024, None) == code
+    assert L.isa_n_keep(ctypes.byref(s)) == -1
+
+
+def test_bad_pointers_and_workspace_rejected(L):
+    s = shape(H=2, N_src=256, N_ctx=256, d=64, block=64)
+    need = L.isa_workspace_size(ctypes.byref(s))
+    buf = (ctypes.c_uint8 * 4096)()
+    p = (ctypes.addressof(buf) + 255) // 256 * 256
+    assert L.isa_preselect_ctx(ctypes.byref(s), None, p, p, p, None, p, need, None) == 1       # null q
+    assert L.isa_preselect_ctx(ctypes.byref(s), p + 2, p, p, p, None, p, need, None) == 1      # misaligned
+    assert L.isa_preselect_ctx(ctypes.byref(s), p, p, p, p, None, p, need - 1, None) == 3      # small ws
+    assert L.isa_preselect_ctx(ctypes.byref(s), p, p, p, None, None, p, need, None) == 1       # kept missing
+    assert L.isa_route_queries(ctypes.byref(s), p, p, None, p, None, p, need, None) == 1       # routed missing
+    assert L.isa_attn_fwd(ctypes.byref(s), p, p, p, p, p, p, None, p, need, None) == 1         # out missing
+    assert L.isa_dense_attn_fwd(1, 1, 128, 80, 0.0, p, p, p, p, p, 256, None) == 2
+    assert L.isa_dense_attn_fwd(1, 1, 128, 64, 0.0, p, p, p, p, p, 8, None) == 3
+    assert L.isa_dense_attn_fwd(1, 1, 0, 64, 0.0, p, p, p, p, p, 256, None) == 1
+
+
+def test_status_strings(L):
+    assert L.isa_status_string(0) == b"ok"
+    assert b"timed out" in L.isa_status_string(5)
+    assert L.isa_status_string(99) == b"unknown status"

@@ -1,0 +1,76 @@
+"""ISA forward on the GPU (through the C ABI) against the float64 oracle,
+stage by stage: saliency and kept context blocks, sharpness and routed /
+Taylor query sets, and the output rows of both attention paths."""
+import numpy as np
+import pytest
+import torch
+
+from sparse_attention_context_b200 import api
+from workloads import CONFIGS, from_torch_bf16
+
+from _parity import check_out, compare_head, inputs, run_stages
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": CONFIGS["tiny"],
+    "small": CONFIGS["small"],
+    # ragged segments, d=128 with 64-token blocks, every partial block in play
+    "ragged128": CONFIGS["tiny"].replace(H=2, d=128, N_src=300, N_ctx=77, block=64, keep=0.6, rho=0.3),
+    "ragged64": CONFIGS["tiny"].replace(H=3, d=64, N_src=1000, N_ctx=1500, block=128, keep=0.4, rho=0.1,
+                                        frame_hw=250),
+    "no_ctx_kept": CONFIGS["tiny"].replace(keep=0.0),
+    "all_taylor": CONFIGS["tiny"].replace(rho=0.0),
+    "all_full": CONFIGS["tiny"].replace(rho=1.0),
+    "keep_all": CONFIGS["tiny"].replace(keep=1.0, rho=0.5),
+    "no_context": CONFIGS["tiny"].replace(N_ctx=0, N_src=300),
+    "ctx_lt_block": CONFIGS["tiny"].replace(N_src=200, N_ctx=50, keep=1.0),
+    "src_lt_block": CONFIGS["tiny"].replace(N_src=30, N_ctx=400, block=128, keep=0.5),
+    "many_tiles": CONFIGS["tiny"].replace(H=1, d=128, N_src=3000, N_ctx=2900, block=128, keep=0.35, rho=0.25),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_isa_stages_match_oracle(cuda_ok, name):
+    cfg = CASES[name]
+    bits, (q, k, v) = inputs(cfg)
+    g = run_stages(cfg, q, k, v)
+    assert g["status"] == 0
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            compare_head(cfg, bits, g, b, h, cfg.keep, cfg.rho)
+    # the one-call entry point runs the same kernels: identical bits
+    out = api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), g["out_t"].view(torch.int16))
+
+
+def test_keep1_rho1_equals_dense_kernel_path(cuda_ok):
+    """keep = rho = 1 reduces ISA to dense attention (up to rounding)."""
+    cfg = CONFIGS["tiny"].replace(keep=1.0, rho=1.0, N_src=300, N_ctx=212)
+    bits, (q, k, v) = inputs(cfg)
+    out = api.isa_forward(q, k, v, cfg.N_src, cfg.block, 1.0, 1.0)
+    dense = api.isa_dense_attn_fwd(q, k, v)
+    torch.cuda.synchronize()
+    check_out(out.double().cpu().numpy(), dense.double().cpu().numpy(), "isa vs dense")
+
+
+@pytest.mark.parametrize("name,heads", [("480p", None), ("720p", [0, 39])])
+def test_isa_full_size_sampled(cuda_ok, name, heads):
+    """Full-size DiT latents.  480p runs all 24 heads in the launch
+    configuration the bench times; 720p runs two of its 40 heads (heads are
+    independent units).  Sets are checked whole, outputs on sampled rows."""
+    cfg = CONFIGS[name]
+    bits, (q, k, v) = inputs(cfg, heads=heads)
+    H = q.shape[1]
+    g = run_stages(cfg.replace(H=H), q, k, v)
+    assert g["status"] == 0
+    rng = np.random.default_rng(7)
+    for h in sorted({0, H - 1}):
+        nr = g["routed"].shape[-1]
+        routed = g["routed"][0, h]
+        taylor = g["taylor"][0, h]
+        rows = np.unique(np.concatenate([
+            rng.choice(routed, min(96, nr), replace=False), rng.choice(taylor, 96, replace=False),
+            [0, cfg.N_src - 1, cfg.N_src, cfg.N - 1]]))
+        compare_head(cfg.replace(H=H), bits, g, 0, h, cfg.keep, cfg.rho, rows=rows)

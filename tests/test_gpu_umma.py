@@ -1,0 +1,26 @@
+"""One-tile checks of the tcgen05 building blocks (K-major S = A B^T and
+MN-major O = P V from TMA-loaded, 128B-swizzled shared memory) against an
+fp32 matrix product computed on the CPU."""
+import pytest
+import torch
+
+from sparse_attention_context_b200 import api
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("d,bn", [(64, 64), (64, 128), (128, 64), (128, 128)])
+def test_umma_tile(cuda_ok, d, bn):
+    g = torch.Generator().manual_seed(d * 1000 + bn)
+    A = torch.randn(128, d, generator=g).bfloat16()
+    B = torch.randn(bn, d, generator=g).bfloat16()
+    P = torch.rand(128, bn, generator=g).bfloat16()
+    V = torch.randn(bn, d, generator=g).bfloat16()
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    S, O = api.isa_selftest_umma(A.cuda(), B.cuda(), P.cuda(), V.cuda(), ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    S_ref = A.double() @ B.double().T
+    O_ref = P.double() @ V.double()
+    assert torch.allclose(S.cpu().double(), S_ref, rtol=1e-5, atol=1e-4), (S.cpu().double() - S_ref).abs().max()
+    assert torch.allclose(O.cpu().double(), O_ref, rtol=1e-5, atol=1e-4), (O.cpu().double() - O_ref).abs().max()
