@@ -22,7 +22,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -77,58 +76,70 @@ def work_model(cfg, kept_tokens_mean):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """Reads SM clocks and clock-event (throttle) reasons through NVML every
+    few milliseconds while the timed region runs (read-only queries)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device, period_s=0.005):
+        self.dev = torch_device
+        self.period = period_s
+        self.sm, self.mx, self.reasons, self.err = [], None, set(), None
+        self._stop = threading.Event()
+        self.h = None
+
+    def _handle(self):
+        import pynvml as nv
+        import torch
+
+        nv.nvmlInit()
+        p = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv, nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv, nv.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
+            try:
+                self.sm.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, attr in self.REASONS.items():
+                    if r & getattr(nv, attr):
+                        self.reasons.add(name)
+            except Exception as e:  # keep timing even if NVML misbehaves
+                self.err = repr(e)
+                return
+            time.sleep(self.period)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            self.nv, self.h = self._handle()
+            self.mx = self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        except Exception:
-            self.proc = None
+        except Exception as e:
+            self.err = repr(e)
+            self.h = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self._stop.set()
+        if self.h is not None:
+            self.t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.sm:
+            return {"sm_mhz": None, "sm_max_mhz": self.mx, "reasons": sorted(self.reasons), "samples": 0,
+                    "source": "nvml", "error": self.err}
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": self.mx, "reasons": sorted(self.reasons),
+                "samples": len(self.sm), "source": "nvml"}
 
 
 def cpu_oracle_ms_per_step(cfg, heads, seed=0):
@@ -173,21 +184,24 @@ def config_dict(cfg, n):
                         f"N_ctx={cfg.N_ctx} block={cfg.block} keep={cfg.keep} rho={cfg.rho}",
             "B": cfg.B, "H": cfg.H, "d": cfg.d, "N_src": cfg.N_src, "N_ctx": cfg.N_ctx, "block": cfg.block,
             "keep": cfg.keep, "rho": cfg.rho, "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
-            "l2": "inputs (747 MB) larger than L2, no flush"}
+            "l2": f"inputs ({3 * cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e6:.0f} MB) larger than the 126 MB L2, no flush"}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="isa", choices=["isa", "reference"])
     ap.add_argument("--config", default="480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--heads", type=int, default=None, help="override H (small profiling captures)")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
+    if args.heads:
+        cfg = cfg.replace(H=args.heads)
     if args.impl == "reference":
         run_reference(args, cfg)
         return
@@ -257,7 +271,7 @@ def main():
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
         t0.record(stream)
         for i in range(args.steps):
             step(i)
@@ -328,10 +342,18 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cms, secs = cpu_oracle_ms_per_step(cfg, [0, cfg.H - 1])
+        # bounded sample: whole heads until ~10 s of CPU work (at most all heads)
+        heads, secs, per_head = [], 0.0, []
+        while secs < 10.0 and len(heads) < cfg.H:
+            h = (len(heads) * 7) % cfg.H
+            _, s1 = cpu_oracle_ms_per_step(cfg, [h])
+            heads.append(h)
+            per_head.append(s1)
+            secs += s1
+        cms = 1e3 * float(np.mean(per_head)) * cfg.B * cfg.H
         cpu = {"value": round(cms, 1), "unit": "ms", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-               "sample": f"heads 0 and {cfg.H - 1} of {cfg.B * cfg.H} ({secs:.1f} s of CPU work), "
-                         f"scaled x{cfg.B * cfg.H / 2:g}"}
+               "sample": f"{len(heads)} of {cfg.B * cfg.H} heads ({secs:.1f} s of CPU work), "
+                         f"scaled x{cfg.B * cfg.H / len(heads):g}"}
 
     launches_per_step = 3 + 3 + (1 if n_route > 0 else 0) + (2 if N - n_route > 0 else 0)
     if rank == 0:
