@@ -6,7 +6,8 @@
  * descriptor shows up as a wrong product rather than as a wrong attention
  * output.  All pointers are device pointers, row-major, 16-byte aligned:
  *   A [128, d] bf16, B [bn, d] bf16      -> S [128, bn] fp32 = A B^T
- *   P [128, bn] bf16, V [bn, d] bf16     -> O [128, d] fp32  = P V
+ *   P [128, bn] bf16, V [bn, d] bf16     -> O [128, d] fp32  = P V  (P from shared memory)
+ *                                        -> O2 [128, d] fp32 = P V  (P from tensor memory)
  * d and bn in {64, 128}.  ws: >= 256 bytes, zeroed; its first int32 receives
  * ISA_ERR_DEVICE_TIMEOUT if a bounded wait expires.  Asynchronous on stream.
  */
@@ -17,7 +18,7 @@
 extern "C" {
 #endif
 int isa_selftest_umma(int d, int bn, const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V,
-                      float* S, float* O, void* ws, void* stream);
+                      float* S, float* O, float* O2, void* ws, void* stream);
 #ifdef __cplusplus
 }
 #endif

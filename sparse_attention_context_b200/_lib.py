@@ -49,7 +49,7 @@ SIGNATURES = {
     "isa_dense_attn_fwd": (_I, [_I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_read_device_status": (_I, [_P, _P]),
     "isa_status_string": (ctypes.c_char_p, [_I]),
-    "isa_selftest_umma": (_I, [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "isa_selftest_umma": (_I, [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 _lib = None

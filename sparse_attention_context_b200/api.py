@@ -174,11 +174,13 @@ def isa_read_device_status(ws, stream=None) -> int:
 
 
 def isa_selftest_umma(A, B, P, V, ws, stream=None):
-    """Test-only: one-tile UMMA products S = A B^T and O = P V (fp32)."""
+    """Test-only: one-tile UMMA products S = A B^T, O = P V (P in shared
+    memory) and O2 = P V (P in tensor memory), all fp32."""
     d, bn = A.shape[1], B.shape[0]
     S = torch.empty((128, bn), dtype=torch.float32, device=A.device)
     O = torch.empty((128, d), dtype=torch.float32, device=A.device)
+    O2 = torch.empty((128, d), dtype=torch.float32, device=A.device)
     rc = lib().isa_selftest_umma(d, bn, A.data_ptr(), B.data_ptr(), P.data_ptr(), V.data_ptr(), S.data_ptr(),
-                                 O.data_ptr(), ws.data_ptr(), _stream(stream))
+                                 O.data_ptr(), O2.data_ptr(), ws.data_ptr(), _stream(stream))
     check("isa_selftest_umma", rc)
-    return S, O
+    return S, O, O2

@@ -2,7 +2,9 @@
 // attention engine: S = A B^T with both operands K-major (A written by
 // threads into the 128B-swizzled layout, B loaded by TMA) and O = P V with
 // V MN-major (loaded by TMA), both accumulated in TMEM and read back with
-// tcgen05.ld.  Exported for the tests only (include/isa_selftest.h).
+// tcgen05.ld; and O2 = P V with P written by threads into TMEM (tcgen05.st,
+// two bf16 per column) and read by the UMMA as its A operand.  Exported for
+// the tests only (include/isa_selftest.h).
 #include "isa.h"
 #include "isa_internal.h"
 #include "isa_selftest.h"
@@ -13,7 +15,8 @@ namespace isa {
 template <int D, int BN>
 __global__ void __launch_bounds__(128, 1)
     umma_probe_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmV,
-                      const uint16_t* A, const uint16_t* P, float* S_out, float* O_out, int* status) {
+                      const uint16_t* A, const uint16_t* P, float* S_out, float* O_out, float* O2_out,
+                      int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -22,9 +25,11 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* sB = sA + A_BYTES;
   uint8_t* sV = sB + B_BYTES;
   uint8_t* sP = sV + B_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + P_BYTES);  // [0] tma, [1] mma
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
-  constexpr int TMEM_COLS = (BN + D) <= 256 ? 256 : 512;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + P_BYTES);  // [0] tma, [1] mma, [2] mma with A in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  // columns: S [0, BN), O [BN, BN+D), P [BN+D, BN+D+BN/2), O2 [.., +D)
+  constexpr int TMEM_COLS = 512;
+  constexpr int PCOL = BN + D, O2COL = BN + D + BN / 2;
   const int tid = threadIdx.x, warp = tid >> 5;
 
   // A (128 x D) and P (128 x BN), K-major, written by threads.
@@ -42,6 +47,7 @@ __global__ void __launch_bounds__(128, 1)
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
+    mbar_init(&bars[2], 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -93,6 +99,42 @@ __global__ void __launch_bounds__(128, 1)
   } else if (tid == 0) {
     atomicCAS(status, 0, ISA_ERR_DEVICE_TIMEOUT);
   }
+  // P into TMEM: lane = row, column c holds P[row][2c] (low half), P[row][2c+1].
+  if (ok) {
+#pragma unroll
+    for (int j = 0; j < BN / 64; ++j) {
+      uint32_t u[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        u[i] = static_cast<uint32_t>(P[row * BN + j * 64 + 2 * i]) |
+               (static_cast<uint32_t>(P[row * BN + j * 64 + 2 * i + 1]) << 16);
+      tmem_st32(tmem + lb + PCOL + j * 32, u);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0) {
+    if (ok)
+      for (int kk = 0; kk < BN / 16; ++kk)
+        umma_bf16_tmem_a(tmem + O2COL, tmem + PCOL + kk * 8, desc_mn_sw128(smem_u32(sV) + kk * 16 * 128, BN * 128),
+                         idesc_bf16(128, D, 1), kk > 0);
+    umma_commit(&bars[2]);
+  }
+  __syncwarp();
+  const bool done2 = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[2], 0, nullptr, kWaitLimitNs) == 0);
+  tc_fence_after();
+  if (ok && done2) {
+    for (int j = 0; j < D / 32; ++j) {
+      uint32_t u[32];
+      tmem_ld32(tmem + lb + O2COL + j * 32, u);
+      tmem_wait_ld();
+      for (int i = 0; i < 32; ++i) O2_out[row * D + j * 32 + i] = __uint_as_float(u[i]);
+    }
+  } else if (tid == 0) {
+    atomicCAS(status, 0, ISA_ERR_DEVICE_TIMEOUT);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -103,27 +145,27 @@ __global__ void __launch_bounds__(128, 1)
 
 template <int D, int BN>
 static int run_probe(const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V, float* S, float* O,
-                     int* status, cudaStream_t st) {
+                     float* O2, int* status, cudaStream_t st) {
   CUtensorMap tmB, tmV;
   if (!make_tmap_bf16(&tmB, B, BN, D, BN) || !make_tmap_bf16(&tmV, V, BN, D, BN)) return ISA_ERR_CUDA;
-  const int smem = 128 * D * 2 + 2 * BN * D * 2 + 128 * BN * 2 + 64 + 1024;
+  const int smem = 128 * D * 2 + 2 * BN * D * 2 + 128 * BN * 2 + 64 + 1024 + 4096;
   auto kern = umma_probe_kernel<D, BN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ISA_ERR_CUDA;
-  kern<<<1, 128, smem, st>>>(tmB, tmV, A, P, S, O, status);
+  kern<<<1, 128, smem, st>>>(tmB, tmV, A, P, S, O, O2, status);
   return cudaGetLastError() == cudaSuccess ? ISA_OK : ISA_ERR_CUDA;
 }
 
 }  // namespace isa
 
 extern "C" int isa_selftest_umma(int d, int bn, const uint16_t* A, const uint16_t* B, const uint16_t* P,
-                                 const uint16_t* V, float* S, float* O, void* ws, void* stream) {
-  if (!A || !B || !P || !V || !S || !O || !ws) return ISA_ERR_INVALID_ARG;
+                                 const uint16_t* V, float* S, float* O, float* O2, void* ws, void* stream) {
+  if (!A || !B || !P || !V || !S || !O || !O2 || !ws) return ISA_ERR_INVALID_ARG;
   int* status = reinterpret_cast<int*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128 && bn == 128) return isa::run_probe<128, 128>(A, B, P, V, S, O, status, st);
-  if (d == 128 && bn == 64) return isa::run_probe<128, 64>(A, B, P, V, S, O, status, st);
-  if (d == 64 && bn == 128) return isa::run_probe<64, 128>(A, B, P, V, S, O, status, st);
-  if (d == 64 && bn == 64) return isa::run_probe<64, 64>(A, B, P, V, S, O, status, st);
+  if (d == 128 && bn == 128) return isa::run_probe<128, 128>(A, B, P, V, S, O, O2, status, st);
+  if (d == 128 && bn == 64) return isa::run_probe<128, 64>(A, B, P, V, S, O, O2, status, st);
+  if (d == 64 && bn == 128) return isa::run_probe<64, 128>(A, B, P, V, S, O, O2, status, st);
+  if (d == 64 && bn == 64) return isa::run_probe<64, 64>(A, B, P, V, S, O, O2, status, st);
   return ISA_ERR_UNSUPPORTED;
 }

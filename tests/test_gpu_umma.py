@@ -1,6 +1,6 @@
 """One-tile checks of the tcgen05 building blocks (K-major S = A B^T and
-MN-major O = P V from TMA-loaded, 128B-swizzled shared memory) against an
-fp32 matrix product computed on the CPU."""
+MN-major O = P V from TMA-loaded, 128B-swizzled shared memory, and P V with
+P as a tensor-memory A operand) against a float64 product on the CPU."""
 import pytest
 import torch
 
@@ -17,10 +17,11 @@ def test_umma_tile(cuda_ok, d, bn):
     P = torch.rand(128, bn, generator=g).bfloat16()
     V = torch.randn(bn, d, generator=g).bfloat16()
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
-    S, O = api.isa_selftest_umma(A.cuda(), B.cuda(), P.cuda(), V.cuda(), ws)
+    S, O, O2 = api.isa_selftest_umma(A.cuda(), B.cuda(), P.cuda(), V.cuda(), ws)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
     S_ref = A.double() @ B.double().T
     O_ref = P.double() @ V.double()
     assert torch.allclose(S.cpu().double(), S_ref, rtol=1e-5, atol=1e-4), (S.cpu().double() - S_ref).abs().max()
     assert torch.allclose(O.cpu().double(), O_ref, rtol=1e-5, atol=1e-4), (O.cpu().double() - O_ref).abs().max()
+    assert torch.allclose(O2.cpu().double(), O_ref, rtol=1e-5, atol=1e-4), (O2.cpu().double() - O_ref).abs().max()
