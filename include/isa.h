@@ -113,6 +113,16 @@ int isa_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, c
                  const int32_t* kept_ctx_idx, const int32_t* routed_idx, const int32_t* taylor_idx,
                  uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Stages 2 and 4 in one pass over q (the fast path of isa_forward): computes
+ * the sharpness of every query and the 0-th order Taylor output of EVERY
+ * row of out [B, H, N, d], then routes exactly as isa_route_queries.  Follow
+ * it with isa_full_attn_fwd on the same out: that overwrites the routed rows
+ * with full attention, leaving the Taylor rows as written here.  Arguments
+ * as in isa_route_queries; sharpness may be NULL. */
+int isa_route_taylor_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
+                         int32_t* routed_idx, int32_t* taylor_idx, float* sharpness, uint16_t* out,
+                         void* ws, size_t ws_bytes, void* stream);
+
 /* Stage 3 alone: full attention for the routed_idx rows of out over every
  * token of every source block and of the kept context blocks (the part of
  * isa_attn_fwd that does not need the block means).  Independent of stage 4:
@@ -127,8 +137,9 @@ int isa_taylor_attn_fwd(const isa_shape* shape, const uint16_t* q, const int32_t
                         const int32_t* taylor_idx, uint16_t* out, void* ws, size_t ws_bytes,
                         void* stream);
 
-/* All four stages in order on one stream, with the kept set and the routed
- * and Taylor index sets held inside ws.  out [B, H, N, d] bf16. */
+/* All four stages in order on one stream (isa_preselect_ctx,
+ * isa_route_taylor_fwd, isa_full_attn_fwd), with the kept set and the
+ * routed and Taylor index sets held inside ws.  out [B, H, N, d] bf16. */
 int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 

@@ -42,6 +42,7 @@ SIGNATURES = {
     "isa_preselect_ctx": (_I, [_SH, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_route_queries": (_I, [_SH, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_attn_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "isa_route_taylor_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_full_attn_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_taylor_attn_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_forward": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),

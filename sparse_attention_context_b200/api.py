@@ -89,6 +89,26 @@ def isa_route_queries(q, kept, shape: IsaShape, ws, routed=None, taylor=None, sh
     return routed, taylor, sharpness
 
 
+def isa_route_taylor_fwd(q, kept, shape: IsaShape, ws, out, routed=None, taylor=None, sharpness=None,
+                         want_sharpness=True, stream=None):
+    """Stages 2 + 4 fused: sharpness, routing, and the Taylor output of every
+    row of `out`.  Returns (routed_idx, taylor_idx, sharpness or None)."""
+    _check_qkv(q, out)
+    B, H, N = shape.B, shape.H, shape.N_src + shape.N_ctx
+    nr = isa_n_route(shape)
+    if routed is None:
+        routed = torch.empty((B, H, nr), dtype=torch.int32, device=q.device)
+    if taylor is None:
+        taylor = torch.empty((B, H, N - nr), dtype=torch.int32, device=q.device)
+    if sharpness is None and want_sharpness:
+        sharpness = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = lib().isa_route_taylor_fwd(ctypes.byref(shape), q.data_ptr(), _ptr(kept) if kept.numel() else None,
+                                    _ptr(routed) if nr > 0 else None, _ptr(taylor) if N - nr > 0 else None,
+                                    _ptr(sharpness), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+    check("isa_route_taylor_fwd", rc)
+    return routed, taylor, sharpness
+
+
 def isa_attn_fwd(q, k, v, kept, routed, taylor, shape: IsaShape, ws, out=None, stream=None):
     """Stages 3 and 4.  Returns out [B,H,N,d] bf16."""
     if out is None:

@@ -1,4 +1,6 @@
-// flash.cu -- the tcgen05 attention engine behind four ISA kernels.
+// flash.cu -- the one-tile tcgen05 attention engine (the SHARP and TAYLOR
+// kernels of the stage-by-stage ABI; the dense, routed-full and fused
+// sharpness+Taylor kernels use the two-tile engine of flash2.cu).
 //
 // One CTA owns 128 query rows of one (b, h) and streams key tiles of BN
 // rows through shared memory (TMA, 128-byte swizzle, two stages).  The
@@ -448,14 +450,8 @@ cudaError_t launch_flash(int D, int BN, int mode, const CUtensorMap& tmK, const 
   if (p.n_rows <= 0 || BH <= 0) return cudaSuccess;
 #define ISA_FLASH_CASE(d_, bn_, m_) \
   if (D == d_ && BN == bn_ && mode == m_) return launch_t<d_, bn_, m_>(tmK, tmV, p, BH, st);
-  ISA_FLASH_CASE(128, 128, MODE_DENSE)
-  ISA_FLASH_CASE(128, 128, MODE_FULL)
-  ISA_FLASH_CASE(128, 64, MODE_FULL)
   ISA_FLASH_CASE(128, 128, MODE_TAYLOR)
   ISA_FLASH_CASE(128, 128, MODE_SHARP)
-  ISA_FLASH_CASE(64, 128, MODE_DENSE)
-  ISA_FLASH_CASE(64, 128, MODE_FULL)
-  ISA_FLASH_CASE(64, 64, MODE_FULL)
   ISA_FLASH_CASE(64, 128, MODE_TAYLOR)
   ISA_FLASH_CASE(64, 128, MODE_SHARP)
 #undef ISA_FLASH_CASE

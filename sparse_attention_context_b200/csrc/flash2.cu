@@ -1,0 +1,485 @@
+// flash2.cu -- two-tile (ping-pong) tcgen05 attention engine.
+//
+// One CTA owns 256 query rows of one (b, h) as two 128-row tiles.  Each tile
+// has its own softmax warpgroup, its own S tile and its own O accumulator in
+// tensor memory; the tensor core alternates between the tiles, so one
+// tile's softmax overlaps the other tile's QK^T and PV products.  The bf16
+// probabilities P are written back into the first BN/2 columns of the
+// tile's own S region (tcgen05.st, two bf16 per column) and consumed from
+// there as the A operand of the PV UMMA; V is the MN-major B operand in
+// 128B-swizzled shared memory.
+//
+// Modes (method: "Lightning Unified Video Editing via In-Context Sparse
+// Attention", abstract):
+//   DENSE  all N keys, contiguous queries (the in-house baseline).
+//   FULL   ISA full attention for routed queries: gathered Q rows, keys of
+//          every source block then of the kept context blocks, one block
+//          per key tile, partial blocks masked by their token count.
+//   FUSED  ISA sharpness and 0-th order Taylor attention in one pass over
+//          every query: logits s*q.Kbar_b + log cnt_b from bf16 q times
+//          Kbar split into bf16 hi + lo parts (two UMMAs, fp32-grade), the
+//          block-mean values as V.  Writes the sharpness of every query and
+//          the Taylor output of every row (routed rows are overwritten by
+//          the FULL pass afterwards).
+//
+// Warps (320 threads): 0-3 softmax of tile 0, 4-7 softmax of tile 1 (thread
+// <-> query row <-> TMEM lane), 8 TMA producer, 9 TMEM allocator + UMMA
+// issuer.  TMEM: S/P of tile i at [i*BN, i*BN+BN), O of tile i at
+// [2*BN + i*D, 2*BN + i*D + D).
+//
+// Ordering: S_i(t+1) overwrites the columns that PV_i(t) reads as P_i(t), so
+// the issuer waits for PV_i(t) to complete (o_done[i]) before issuing
+// S_i(t+1); in between it issues PV of the other tile, so the tensor pipe
+// stays fed.  A softmax warpgroup that sees S_i(t) may therefore touch O_i
+// (rescale) and overwrite the S_i columns with P_i(t) without further waits.
+// Every mbarrier wait is bounded (status word + CTA abort flag, as in
+// flash.cu).
+#include <cmath>
+
+#include "isa_internal.h"
+#include "tc_ptx.cuh"
+
+namespace isa {
+
+template <int D, int BN, int MODE>
+struct Attn2Cfg {
+  static constexpr int TILE = 128;
+  static constexpr bool kFused = MODE == MODE_FUSED;
+  static constexpr bool kTmaQ = MODE != MODE_FULL;  // contiguous query rows
+  static constexpr int Q_BYTES = TILE * D * 2;      // one tile
+  static constexpr int KT_BYTES = BN * D * 2;       // one key (or value) tile
+  static constexpr int NKT = kFused ? 3 : 2;        // tiles per stage: K[,Klo],V
+  static constexpr int STAGE_BYTES = NKT * KT_BYTES;
+  static constexpr int BUDGET = 225 * 1024;
+  static constexpr int ST_FIT = (BUDGET - 2 * Q_BYTES - 1024 - 256) / STAGE_BYTES;
+  static constexpr int STAGES = ST_FIT >= 3 ? 3 : (ST_FIT >= 2 ? 2 : 1);
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = 2 * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE_BYTES;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 320;
+  static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
+  static_assert(ST_FIT >= 1, "shared memory budget");
+};
+
+struct Attn2Bars {
+  uint64_t q_full[2];
+  uint64_t k_full[3];
+  uint64_t v_full[3];
+  uint64_t kv_empty[3];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t teardown;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void raise2(Attn2Bars* bars, const FlashParams& p) {
+  *reinterpret_cast<volatile int*>(&bars->abort) = 1;
+  if (p.status != nullptr) atomicCAS(p.status, 0, 5 /* ISA_ERR_DEVICE_TIMEOUT */);
+}
+__device__ __forceinline__ bool w1(uint64_t* bar, uint32_t par, Attn2Bars* bars, const FlashParams& p) {
+  const int r = mbar_wait_bounded(bar, par, reinterpret_cast<volatile int*>(&bars->abort), kWaitLimitNs);
+  if (r == 2) raise2(bars, p);
+  return r == 0;
+}
+__device__ __forceinline__ bool wwarp(uint64_t* bar, uint32_t par, Attn2Bars* bars, const FlashParams& p) {
+  const bool ok = w1(bar, par, bars, p);
+  return __all_sync(0xffffffffu, ok);
+}
+template <int N>
+__device__ __forceinline__ void regs_after(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+template <int BN, int MODE>
+__device__ __forceinline__ int kv_row(const FlashParams& p, int bh, int t) {
+  if constexpr (MODE == MODE_FULL) {
+    const int start = (t < p.nSB) ? t * p.blk
+                                  : p.N_src + __ldg(p.kept_ctx + static_cast<size_t>(bh) * p.n_keep + (t - p.nSB)) * p.blk;
+    return bh * p.N + start;
+  } else if constexpr (MODE == MODE_DENSE) {
+    return bh * p.N + t * BN;
+  } else {
+    return bh * p.kv_rows_per_head + t * BN;
+  }
+}
+template <int BN, int MODE>
+__device__ __forceinline__ int kv_count(const FlashParams& p, int bh, int t) {
+  if constexpr (MODE == MODE_FULL) {
+    if (t < p.nSB) return min(p.blk, p.N_src - t * p.blk);
+    const int c = __ldg(p.kept_ctx + static_cast<size_t>(bh) * p.n_keep + (t - p.nSB));
+    return min(p.blk, p.N_ctx - c * p.blk);
+  } else if constexpr (MODE == MODE_DENSE) {
+    return min(BN, p.N - t * BN);
+  } else {
+    return BN;
+  }
+}
+
+template <int D, int BN, int MODE>
+__global__ void __maxnreg__(200)
+    attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmK2, const __grid_constant__ CUtensorMap tmV,
+                 const FlashParams p) {
+  using C = Attn2Cfg<D, BN, MODE>;
+  constexpr int ST = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  Attn2Bars* bars = reinterpret_cast<Attn2Bars*>(smem + C::OFF_BAR);
+  const uint32_t aQ = smem_u32(smem + C::OFF_Q);
+  const uint32_t aKV = smem_u32(smem + C::OFF_KV);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y;
+  const int row0 = blockIdx.x * 256;
+  const int nT = p.n_kv_tiles;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q_full[i], C::kTmaQ ? 1 : 128);
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_done[i], 1);
+    }
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->teardown, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    if constexpr (C::kTmaQ) tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    if constexpr (C::kFused) tma_prefetch_desc(&tmK2);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      if constexpr (C::kTmaQ) {
+        for (int i = 0; i < 2; ++i) {
+          mbar_arrive_expect_tx(&bars->q_full[i], C::Q_BYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(smem + C::OFF_Q + i * C::Q_BYTES + c * (128 * 128), &tmQ, &bars->q_full[i], c * 64,
+                        bh * p.N + row0 + i * 128);
+        }
+      }
+      int issued = 0;
+      for (int t = 0; t < nT; ++t) {
+        const int st = t % ST;
+        if (t >= ST && !w1(&bars->kv_empty[st], ((t / ST) - 1) & 1, bars, p)) break;
+        const int r = kv_row<BN, MODE>(p, bh, t);
+        uint8_t* base = smem + C::OFF_KV + st * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(&bars->k_full[st], (C::kFused ? 2 : 1) * C::KT_BYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tma_load_2d(base + c * (BN * 128), &tmK, &bars->k_full[st], c * 64, r);
+        if constexpr (C::kFused) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(base + C::KT_BYTES + c * (BN * 128), &tmK2, &bars->k_full[st], c * 64, r);
+        }
+        uint8_t* vb = base + (C::NKT - 1) * C::KT_BYTES;
+        mbar_arrive_expect_tx(&bars->v_full[st], C::KT_BYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tma_load_2d(vb + c * (BN * 128), &tmV, &bars->v_full[st], c * 64, r);
+        issued = t + 1;
+      }
+      for (int t = issued > ST ? issued - ST : 0; t < issued; ++t) {  // drain own copies
+        const int st = t % ST;
+        const uint32_t par = (t / ST) & 1;
+        mbar_wait_bounded(&bars->k_full[st], par, nullptr, kWaitLimitNs);
+        mbar_wait_bounded(&bars->v_full[st], par, nullptr, kWaitLimitNs);
+      }
+      if constexpr (C::kTmaQ) {
+        mbar_wait_bounded(&bars->q_full[0], 0, nullptr, kWaitLimitNs);
+        mbar_wait_bounded(&bars->q_full[1], 0, nullptr, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDS = idesc_bf16(128, BN, 0);
+      constexpr uint32_t IDO = idesc_bf16(128, D, 1);
+      bool ok = w1(&bars->q_full[0], 0, bars, p) && w1(&bars->q_full[1], 0, bars, p);
+      tc_fence_after();
+      auto issue_S = [&](int i, int t) {
+        const int st = t % ST;
+        const uint32_t kb = aKV + st * C::STAGE_BYTES;
+        const uint32_t qa = aQ + i * C::Q_BYTES;
+        const uint32_t dS = tmem + i * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                    desc_k_sw128(kb + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, kk > 0 ? 1u : 0u);
+        if constexpr (C::kFused) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                      desc_k_sw128(kb + C::KT_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, 1u);
+        }
+        umma_commit(&bars->s_full[i]);
+      };
+      auto issue_PV = [&](int i, int t) {
+        const int st = t % ST;
+        const uint32_t vb = aKV + st * C::STAGE_BYTES + (C::NKT - 1) * C::KT_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_tmem_a(tmem + 2 * BN + i * D, tmem + i * BN + kk * 8, desc_mn_sw128(vb + kk * 16 * 128, BN * 128),
+                           IDO, (t > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bars->o_done[i]);
+      };
+      if (ok && nT > 0) {
+        ok = w1(&bars->k_full[0], 0, bars, p);
+        if (ok) {
+          tc_fence_after();
+          issue_S(0, 0);
+          issue_S(1, 0);
+        }
+      }
+      for (int t = 0; ok && t < nT; ++t) {
+        const int st = t % ST;
+        const uint32_t ph = t & 1;
+        if (!(ok = w1(&bars->v_full[st], (t / ST) & 1, bars, p))) break;
+        if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
+        tc_fence_after();
+        issue_PV(0, t);
+        if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
+        tc_fence_after();
+        issue_PV(1, t);
+        umma_commit(&bars->kv_empty[st]);
+        if (t + 1 < nT) {
+          const int st1 = (t + 1) % ST;
+          if (!(ok = w1(&bars->k_full[st1], ((t + 1) / ST) & 1, bars, p))) break;
+          if (!(ok = w1(&bars->o_done[0], ph, bars, p))) break;
+          tc_fence_after();
+          issue_S(0, t + 1);
+          if (!(ok = w1(&bars->o_done[1], ph, bars, p))) break;
+          tc_fence_after();
+          issue_S(1, t + 1);
+        }
+      }
+      umma_commit(&bars->teardown);
+      mbar_wait_bounded(&bars->teardown, 0, nullptr, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------ softmax warpgroup of tile i
+    const int i = warp >> 2;
+    const int r = tid & 127;
+    const int g = row0 + i * 128 + r;  // query row within the launch's row list
+    if constexpr (!C::kTmaQ) {
+      constexpr int CPR = D / 8;
+      uint4 vals[CPR];
+#pragma unroll
+      for (int it = 0; it < CPR; ++it) {
+        const int c = it * 128 + r;
+        const int row = c / CPR, ch = c % CPR;
+        const int gg = row0 + i * 128 + row;
+        vals[it] = make_uint4(0u, 0u, 0u, 0u);
+        if (gg < p.n_rows) {
+          const int src = p.row_idx ? __ldg(p.row_idx + static_cast<size_t>(bh) * p.n_rows + gg) : gg;
+          if (static_cast<unsigned>(src) < static_cast<unsigned>(p.N))
+            vals[it] = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.N + src) * D + ch * 8));
+          else if (p.status != nullptr)
+            atomicCAS(p.status, 0, 1 /* ISA_ERR_INVALID_ARG: index out of range, row skipped */);
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < CPR; ++it) {
+        const int c = it * 128 + r;
+        const int row = c / CPR, ch = c % CPR;
+        st_shared_v4(aQ + i * C::Q_BYTES + (ch >> 3) * (128 * 128) + sw128(row, ch & 7), vals[it].x, vals[it].y,
+                     vals[it].z, vals[it].w);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->q_full[i]);
+    }
+
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t sS = tmem + lane_base + i * BN;
+    const uint32_t sO = tmem + lane_base + 2 * BN + i * D;
+    float m = -INFINITY, l = 0.f, mx = -INFINITY;
+    bool ok = true;
+    if (p.inject != nullptr && (__ldg(p.inject) & 1)) {  // test hook: behave as if S never arrived
+      raise2(bars, p);
+      ok = false;
+    }
+    for (int t = 0; ok && t < nT; ++t) {
+      if (!(ok = wwarp(&bars->s_full[i], t & 1, bars, p))) break;
+      tc_fence_after();
+      float x[BN];
+      {
+        uint32_t u[BN / 32][32];
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) tmem_ld32(sS + j * 32, u[j]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) {
+          regs_after(u[j]);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[j * 32 + c] = __uint_as_float(u[j][c]);
+        }
+      }
+      // logits in log2 units
+      if constexpr (C::kFused) {
+        const float4* bp = reinterpret_cast<const float4*>(p.bias2 + static_cast<size_t>(bh) * p.kv_rows_per_head + t * BN);
+#pragma unroll
+        for (int c4 = 0; c4 < BN / 4; ++c4) {
+          const float4 b = __ldg(bp + c4);
+          x[4 * c4 + 0] = fmaf(x[4 * c4 + 0], p.scale_log2, b.x);
+          x[4 * c4 + 1] = fmaf(x[4 * c4 + 1], p.scale_log2, b.y);
+          x[4 * c4 + 2] = fmaf(x[4 * c4 + 2], p.scale_log2, b.z);
+          x[4 * c4 + 3] = fmaf(x[4 * c4 + 3], p.scale_log2, b.w);
+        }
+      } else {
+        const int valid = kv_count<BN, MODE>(p, bh, t);
+        if (valid < BN) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c >= valid) x[c] = -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < BN; ++c) x[c] *= p.scale_log2;
+      }
+      float mt;
+      {
+        float pm[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pm[k] = x[k];
+#pragma unroll
+        for (int c = 8; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
+        mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      }
+      mx = fmaxf(mx, mt);
+      const float m_new = fmaxf(m, mt);
+      // Rescale only when the running maximum grew by more than 2^8: the
+      // stale reference keeps every p <= 256, exact after the final 1/l.
+      const bool need = m_new > m + 8.0f;
+      if (t > 0 && __any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2(m - m_new) : 1.f;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          uint32_t u[32];
+          tmem_ld32(sO + j * 32, u);
+          tmem_wait_ld();
+          regs_after(u);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+          tmem_st32(sO + j * 32, u);
+        }
+      }
+      if (need) {
+        l *= ex2(m - m_new);
+        m = m_new;
+      }
+      const float mref = (m == -INFINITY) ? 0.f : m;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < BN / 32; ++j) {  // 32 probabilities -> 16 packed columns
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float e0 = ex2(x[j * 32 + 2 * c] - mref);
+          const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
+          ps[(2 * c) & 7] += e0;
+          ps[(2 * c + 1) & 7] += e1;
+          w[c] = pack_bf16(e0, e1);
+        }
+        tmem_st16(sS + j * 16, w);
+      }
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[i]);
+    }
+
+    const bool valid_row = g < p.n_rows;
+    if (ok && nT > 0 && wwarp(&bars->o_done[i], (nT - 1) & 1, bars, p)) {
+      tc_fence_after();
+      int dst = valid_row ? (p.row_idx ? __ldg(p.row_idx + static_cast<size_t>(bh) * p.n_rows + g) : g) : 0;
+      const bool store = valid_row && static_cast<unsigned>(dst) < static_cast<unsigned>(p.N);
+      if (!store) dst = 0;
+      if constexpr (C::kFused) {
+        // sharpness = max_b softmax_b = 2^(mx - m) / l (l is relative to m)
+        if (store) p.sharp[static_cast<size_t>(bh) * p.N + dst] = ex2(mx - m) / l;
+      }
+      uint16_t* orow = p.out + (static_cast<size_t>(bh) * p.N + dst) * D;
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        uint32_t u[32];
+        tmem_ld32(sO + j * 32, u);
+        tmem_wait_ld();
+        regs_after(u);
+        if (store) {
+          uint4* o4 = reinterpret_cast<uint4*>(orow + j * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(u[8 * q4 + 0]) * inv, __uint_as_float(u[8 * q4 + 1]) * inv);
+            w.y = pack_bf16(__uint_as_float(u[8 * q4 + 2]) * inv, __uint_as_float(u[8 * q4 + 3]) * inv);
+            w.z = pack_bf16(__uint_as_float(u[8 * q4 + 4]) * inv, __uint_as_float(u[8 * q4 + 5]) * inv);
+            w.w = pack_bf16(__uint_as_float(u[8 * q4 + 6]) * inv, __uint_as_float(u[8 * q4 + 7]) * inv);
+            o4[q4] = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, int BN, int MODE>
+static cudaError_t launch2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmK2,
+                             const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st) {
+  using C = Attn2Cfg<D, BN, MODE>;
+  auto kern = attn2_kernel<D, BN, MODE>;
+  const int smem = C::SMEM < 116 * 1024 ? 116 * 1024 : C::SMEM;  // one CTA per SM (all 512 TMEM columns)
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((p.n_rows + 255) / 256, BH);
+  kern<<<grid, C::THREADS, smem, st>>>(tmQ, tmK, tmK2, tmV, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                         const CUtensorMap& tmK2, const CUtensorMap& tmV, const FlashParams& p, int BH,
+                         cudaStream_t st) {
+  if (p.n_rows <= 0 || BH <= 0) return cudaSuccess;
+#define ISA_ATTN2_CASE(d_, bn_, m_) \
+  if (D == d_ && BN == bn_ && mode == m_) return launch2_t<d_, bn_, m_>(tmQ, tmK, tmK2, tmV, p, BH, st);
+  ISA_ATTN2_CASE(128, 128, MODE_DENSE)
+  ISA_ATTN2_CASE(128, 128, MODE_FULL)
+  ISA_ATTN2_CASE(128, 64, MODE_FULL)
+  ISA_ATTN2_CASE(128, 128, MODE_FUSED)
+  ISA_ATTN2_CASE(64, 128, MODE_DENSE)
+  ISA_ATTN2_CASE(64, 128, MODE_FULL)
+  ISA_ATTN2_CASE(64, 64, MODE_FULL)
+  ISA_ATTN2_CASE(64, 128, MODE_FUSED)
+#undef ISA_ATTN2_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace isa

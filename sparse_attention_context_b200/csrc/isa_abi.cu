@@ -199,6 +199,35 @@ int run_route(const Ctx& c, const uint16_t* q, const int32_t* kept, int32_t* rou
   return cuda_status(e);
 }
 
+// Stages 2 and 4 in one pass over q: sharpness and the Taylor output of
+// every row (fused kernel), then routing.
+int run_route_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, int32_t* routed, int32_t* taylor,
+                     float* sharp_user, uint16_t* out) {
+  const Dims& d = c.d;
+  int rc = run_build_kept(c, kept);
+  if (rc != ISA_OK) return rc;
+  CUtensorMap tmQ, tmHi, tmLo, tmVb;
+  const uint64_t kv_rows = static_cast<uint64_t>(d.BH) * d.nKpad;
+  if (!make_tmap_bf16(&tmQ, q, static_cast<uint64_t>(d.BH) * d.N, d.d, 128) ||
+      !make_tmap_bf16(&tmHi, at<uint16_t>(c.ws, c.L.Khi), kv_rows, d.d, 128) ||
+      !make_tmap_bf16(&tmLo, at<uint16_t>(c.ws, c.L.Klo), kv_rows, d.d, 128) ||
+      !make_tmap_bf16(&tmVb, at<uint16_t>(c.ws, c.L.Vb), kv_rows, d.d, 128))
+    return ISA_ERR_CUDA;
+  float* sharp = sharp_user ? sharp_user : at<float>(c.ws, c.L.sharp);
+  FlashParams p = base_params(c);
+  p.q = q;
+  p.out = out;
+  p.sharp = sharp;
+  p.row_idx = nullptr;
+  p.n_rows = d.N;
+  p.n_kv_tiles = d.nKpad / 128;
+  p.kv_rows_per_head = d.nKpad;
+  p.bias2 = at<float>(c.ws, c.L.bias2);
+  cudaError_t e = launch_attn2(d.d, 128, MODE_FUSED, tmQ, tmHi, tmLo, tmVb, p, d.BH, c.st);
+  if (e == cudaSuccess) e = launch_route(sharp, routed, taylor, d.BH, d.N, d.n_route, c.status(), c.st);
+  return cuda_status(e);
+}
+
 int run_full(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kept,
              const int32_t* routed, uint16_t* out) {
   const Dims& d = c.d;
@@ -216,7 +245,7 @@ int run_full(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t*
     p.kept_ctx = kept;
     p.n_kv_tiles = d.nSB + d.n_keep;
     p.kv_rows_per_head = d.N;
-    e = launch_flash(d.d, d.blk, MODE_FULL, tmK, tmV, p, d.BH, c.st);
+    e = launch_attn2(d.d, d.blk, MODE_FULL, tmK /* Q is gathered by threads */, tmK, tmK, tmV, p, d.BH, c.st);
   }
   return cuda_status(e);
 }
@@ -345,6 +374,20 @@ int isa_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, c
   return run_attn(c, q, k, v, kept_ctx_idx, routed_idx, taylor_idx, out, true);
 }
 
+int isa_route_taylor_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
+                         int32_t* routed_idx, int32_t* taylor_idx, float* sharpness, uint16_t* out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q, out})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_route > 0 && (routed_idx == nullptr || !aligned16(routed_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.N - c.d.n_route > 0 && (taylor_idx == nullptr || !aligned16(taylor_idx))) return ISA_ERR_INVALID_ARG;
+  if (sharpness != nullptr && !aligned16(sharpness)) return ISA_ERR_INVALID_ARG;
+  return run_route_taylor(c, q, kept_ctx_idx, routed_idx, taylor_idx, sharpness, out);
+}
+
 int isa_full_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                       const int32_t* kept_ctx_idx, const int32_t* routed_idx, uint16_t* out, void* ws,
                       size_t ws_bytes, void* stream) {
@@ -378,8 +421,8 @@ int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, co
   int32_t* routed = at<int32_t>(ws, c.L.routed);
   int32_t* taylor = at<int32_t>(ws, c.L.taylor);
   rc = run_preselect(c, q, k, v, kept, nullptr);
-  if (rc == ISA_OK) rc = run_route(c, q, kept, routed, taylor, nullptr);
-  if (rc == ISA_OK) rc = run_attn(c, q, k, v, kept, routed, taylor, out, false);
+  if (rc == ISA_OK) rc = run_route_taylor(c, q, kept, routed, taylor, nullptr, out);
+  if (rc == ISA_OK) rc = run_full(c, q, k, v, kept, routed, out);
   return rc;
 }
 
@@ -394,8 +437,9 @@ int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* 
   if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
   int rc = check_ws(ws, ws_bytes, kCtlBytes);
   if (rc != ISA_OK) return rc;
-  CUtensorMap tmK, tmV;
-  if (!make_tmap_bf16(&tmK, k, static_cast<uint64_t>(BH) * N, d, 128) ||
+  CUtensorMap tmQ, tmK, tmV;
+  if (!make_tmap_bf16(&tmQ, q, static_cast<uint64_t>(BH) * N, d, 128) ||
+      !make_tmap_bf16(&tmK, k, static_cast<uint64_t>(BH) * N, d, 128) ||
       !make_tmap_bf16(&tmV, v, static_cast<uint64_t>(BH) * N, d, 128))
     return ISA_ERR_CUDA;
   FlashParams p{};
@@ -409,7 +453,7 @@ int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* 
   p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d))) * 1.4426950408889634f;
   p.status = at<int>(ws, kStatusOffset);
   p.inject = at<int>(ws, kInjectOffset);
-  return cuda_status(launch_flash(d, 128, MODE_DENSE, tmK, tmV, p, static_cast<int>(BH),
+  return cuda_status(launch_attn2(d, 128, MODE_DENSE, tmQ, tmK, tmK, tmV, p, static_cast<int>(BH),
                                   static_cast<cudaStream_t>(stream)));
 }
 

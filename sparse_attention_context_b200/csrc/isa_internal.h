@@ -15,7 +15,7 @@ constexpr int kTopkCap = 4096;     // max context blocks the top-k sort holds
 constexpr int kSalRows = 16;       // query blocks per saliency CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
-enum FlashMode { MODE_DENSE = 0, MODE_FULL = 1, MODE_TAYLOR = 2, MODE_SHARP = 3 };
+enum FlashMode { MODE_DENSE = 0, MODE_FULL = 1, MODE_TAYLOR = 2, MODE_SHARP = 3, MODE_FUSED = 4 };
 
 // Arguments of the tcgen05 attention engine (one CTA = 128 query rows of
 // one (b, h); grid = (ceil(n_rows/128), B*H)).
@@ -42,8 +42,15 @@ struct FlashParams {
 // box_rows rows, 128-byte swizzle.  Returns false if encoding fails.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows);
 
+// One-tile engine (flash.cu): SHARP and TAYLOR modes; grid (ceil(n_rows/128), BH).
 cudaError_t launch_flash(int D, int BN, int mode, const CUtensorMap& tmK, const CUtensorMap& tmV,
                          const FlashParams& p, int BH, cudaStream_t st);
+// Two-tile engine (flash2.cu): DENSE, FULL and FUSED modes; grid
+// (ceil(n_rows/256), BH).  tmQ is read in DENSE / FUSED (contiguous rows,
+// box 64 x 128); tmK2 (the lo part of the split block means) only in FUSED.
+cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                         const CUtensorMap& tmK2, const CUtensorMap& tmV, const FlashParams& p, int BH,
+                         cudaStream_t st);
 
 // Stage-1 kernels.
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,

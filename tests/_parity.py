@@ -68,6 +68,23 @@ def run_stages(cfg: Config, q, k, v, keep=None, rho=None):
                 out=bf16_bits_to_f64(from_torch_bf16(out)), out_t=out, status=status)
 
 
+def run_fused(cfg: Config, q, k, v, keep=None, rho=None):
+    """The isa_forward path, one call per stage: pre-selection, the fused
+    sharpness + Taylor pass with routing, then full attention."""
+    keep = cfg.keep if keep is None else keep
+    rho = cfg.rho if rho is None else rho
+    shape = api.make_shape(q, cfg.N_src, cfg.block, keep, rho)
+    ws = api.new_workspace(shape)
+    out = torch.empty_like(q)
+    kept, sal = api.isa_preselect_ctx(q, k, v, shape, ws)
+    routed, taylor, sharp = api.isa_route_taylor_fwd(q, kept, shape, ws, out)
+    api.isa_full_attn_fwd(q, k, v, kept, routed, shape, ws, out)
+    status = api.isa_read_device_status(ws)
+    return dict(shape=shape, ws=ws, kept=kept.cpu().numpy(), sal=None if sal is None else sal.cpu().numpy(),
+                routed=routed.cpu().numpy(), taylor=taylor.cpu().numpy(), sharp=sharp.cpu().numpy(),
+                out=bf16_bits_to_f64(from_torch_bf16(out)), out_t=out, status=status)
+
+
 def compare_head(cfg: Config, bits, g, b, h, keep, rho, rows=None):
     """Check one (b, h) of a GPU run `g` against the oracle, stage by stage.
     `rows` restricts the output comparison to a sample of rows."""

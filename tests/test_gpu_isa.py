@@ -8,7 +8,7 @@ import torch
 from sparse_attention_context_b200 import api
 from workloads import CONFIGS, from_torch_bf16
 
-from _parity import check_out, compare_head, inputs, run_stages
+from _parity import check_out, check_set, compare_head, inputs, run_fused, run_stages
 
 pytestmark = pytest.mark.gpu
 
@@ -32,17 +32,22 @@ CASES = {
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_isa_stages_match_oracle(cuda_ok, name):
+    """Stage-by-stage ABI (isa_route_queries, isa_attn_fwd) and the fused
+    path of isa_forward (isa_route_taylor_fwd + isa_full_attn_fwd), each
+    against the oracle."""
     cfg = CASES[name]
     bits, (q, k, v) = inputs(cfg)
     g = run_stages(cfg, q, k, v)
-    assert g["status"] == 0
+    f = run_fused(cfg, q, k, v)
+    assert g["status"] == 0 and f["status"] == 0
     for b in range(cfg.B):
         for h in range(cfg.H):
             compare_head(cfg, bits, g, b, h, cfg.keep, cfg.rho)
-    # the one-call entry point runs the same kernels: identical bits
+            compare_head(cfg, bits, f, b, h, cfg.keep, cfg.rho)
+    # the one-call entry point runs the fused path's kernels: identical bits
     out = api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     torch.cuda.synchronize()
-    assert torch.equal(out.view(torch.int16), g["out_t"].view(torch.int16))
+    assert torch.equal(out.view(torch.int16), f["out_t"].view(torch.int16))
 
 
 def test_keep1_rho1_equals_dense_kernel_path(cuda_ok):
@@ -57,13 +62,14 @@ def test_keep1_rho1_equals_dense_kernel_path(cuda_ok):
 
 @pytest.mark.parametrize("name,heads", [("480p", None), ("720p", [0, 39])])
 def test_isa_full_size_sampled(cuda_ok, name, heads):
-    """Full-size DiT latents.  480p runs all 24 heads in the launch
-    configuration the bench times; 720p runs two of its 40 heads (heads are
-    independent units).  Sets are checked whole, outputs on sampled rows."""
+    """Full-size DiT latents through the fused path that isa_forward and the
+    bench run.  480p runs all 24 heads in the launch configuration the bench
+    times; 720p runs two of its 40 heads (heads are independent units).
+    Sets are checked whole, outputs on sampled rows."""
     cfg = CONFIGS[name]
     bits, (q, k, v) = inputs(cfg, heads=heads)
     H = q.shape[1]
-    g = run_stages(cfg.replace(H=H), q, k, v)
+    g = run_fused(cfg.replace(H=H), q, k, v)
     assert g["status"] == 0
     rng = np.random.default_rng(7)
     for h in sorted({0, H - 1}):
