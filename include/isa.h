@@ -159,6 +159,10 @@ int isa_read_device_status(void* ws, void* stream);
 /* Static description of a status code. */
 const char* isa_status_string(int status);
 
+/* Description of the CUDA error behind the calling thread's most recent
+ * ISA_ERR_CUDA (a static string owned by the CUDA runtime). */
+const char* isa_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

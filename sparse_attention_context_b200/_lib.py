@@ -23,8 +23,8 @@ class IsaShape(ctypes.Structure):
 
 
 class IsaError(RuntimeError):
-    def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn} failed: {STATUS.get(code, code)} ({code})")
+    def __init__(self, fn: str, code: int, detail: str = ""):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)} ({code}){': ' + detail if detail else ''}")
         self.code = code
 
 
@@ -50,6 +50,7 @@ SIGNATURES = {
     "isa_dense_attn_fwd": (_I, [_I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_read_device_status": (_I, [_P, _P]),
     "isa_status_string": (ctypes.c_char_p, [_I]),
+    "isa_last_error": (ctypes.c_char_p, []),
     "isa_selftest_umma": (_I, [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
@@ -73,4 +74,5 @@ def lib():
 
 def check(fn: str, code: int) -> None:
     if code != ISA_OK:
-        raise IsaError(fn, code)
+        detail = lib().isa_last_error().decode() if code == 4 else ""
+        raise IsaError(fn, code, detail)

@@ -56,7 +56,7 @@ struct Attn2Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE_BYTES;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + runtime key-bias table (FUSED)
   static constexpr int THREADS = 320;
   static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
   static_assert(ST_FIT >= 1, "shared memory budget");
@@ -120,7 +120,7 @@ __device__ __forceinline__ int kv_count(const FlashParams& p, int bh, int t) {
 }
 
 template <int D, int BN, int MODE>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(320, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmK2, const __grid_constant__ CUtensorMap tmV,
                  const FlashParams p) {
@@ -320,51 +320,71 @@ __global__ void __maxnreg__(200)
       raise2(bars, p);
       ok = false;
     }
+    // FUSED: the head's log2(cnt) key biases (-inf padding) in shared memory.
+    float* sBias = reinterpret_cast<float*>(smem + C::OFF_BAR + 256);
+    if constexpr (C::kFused) {
+      for (int c = tid; c < p.kv_rows_per_head; c += 256)
+        sBias[c] = __ldg(p.bias2 + static_cast<size_t>(bh) * p.kv_rows_per_head + c);
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // the two softmax warpgroups only
+    }
+    // Softmax on 64-column halves of the S tile (a second tcgen05.ld of S
+    // replaces keeping all BN logits in registers: 10 warps per SM leave
+    // 168 registers per thread).
+    constexpr int NH = BN / 64;
     for (int t = 0; ok && t < nT; ++t) {
       if (!(ok = wwarp(&bars->s_full[i], t & 1, bars, p))) break;
       tc_fence_after();
-      float x[BN];
-      {
-        uint32_t u[BN / 32][32];
+      const int valid = kv_count<BN, MODE>(p, bh, t);
+      const float* bias = C::kFused ? sBias + t * BN : nullptr;
+      // logits of half h, in log2 units (-inf outside the tile's tokens)
+      auto load_half = [&](int h, float (&x)[64]) {
+        if constexpr (C::kFused) {
+          // 32 columns at a time: the bias reads stay out of the TMEM registers' way
 #pragma unroll
-        for (int j = 0; j < BN / 32; ++j) tmem_ld32(sS + j * 32, u[j]);
-        tmem_wait_ld();
+          for (int q2 = 0; q2 < 2; ++q2) {
+            uint32_t u[32];
+            tmem_ld32(sS + h * 64 + q2 * 32, u);
+            tmem_wait_ld();
+            regs_after(u);
+            const float4* bp = reinterpret_cast<const float4*>(bias + h * 64 + q2 * 32);
 #pragma unroll
-        for (int j = 0; j < BN / 32; ++j) {
-          regs_after(u[j]);
+            for (int c4 = 0; c4 < 8; ++c4) {
+              const float4 b = bp[c4];
+              const int c = 4 * c4;
+              x[q2 * 32 + c + 0] = fmaf(__uint_as_float(u[c + 0]), p.scale_log2, b.x);
+              x[q2 * 32 + c + 1] = fmaf(__uint_as_float(u[c + 1]), p.scale_log2, b.y);
+              x[q2 * 32 + c + 2] = fmaf(__uint_as_float(u[c + 2]), p.scale_log2, b.z);
+              x[q2 * 32 + c + 3] = fmaf(__uint_as_float(u[c + 3]), p.scale_log2, b.w);
+            }
+          }
+        } else {
+          uint32_t u[2][32];
+          tmem_ld32(sS + h * 64, u[0]);
+          tmem_ld32(sS + h * 64 + 32, u[1]);
+          tmem_wait_ld();
+          regs_after(u[0]);
+          regs_after(u[1]);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) x[j * 32 + c] = __uint_as_float(u[j][c]);
+          for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(u[c >> 5][c & 31]) * p.scale_log2;
+          if (valid < (h + 1) * 64) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (h * 64 + c >= valid) x[c] = -INFINITY;
+          }
         }
-      }
-      // logits in log2 units
-      if constexpr (C::kFused) {
-        const float4* bp = reinterpret_cast<const float4*>(p.bias2 + static_cast<size_t>(bh) * p.kv_rows_per_head + t * BN);
+      };
+      float mt = -INFINITY;
 #pragma unroll
-        for (int c4 = 0; c4 < BN / 4; ++c4) {
-          const float4 b = __ldg(bp + c4);
-          x[4 * c4 + 0] = fmaf(x[4 * c4 + 0], p.scale_log2, b.x);
-          x[4 * c4 + 1] = fmaf(x[4 * c4 + 1], p.scale_log2, b.y);
-          x[4 * c4 + 2] = fmaf(x[4 * c4 + 2], p.scale_log2, b.z);
-          x[4 * c4 + 3] = fmaf(x[4 * c4 + 3], p.scale_log2, b.w);
-        }
-      } else {
-        const int valid = kv_count<BN, MODE>(p, bh, t);
-        if (valid < BN) {
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c >= valid) x[c] = -INFINITY;
-        }
-#pragma unroll
-        for (int c = 0; c < BN; ++c) x[c] *= p.scale_log2;
-      }
-      float mt;
-      {
+      for (int h = 0; h < NH; ++h) {
+        float x[64];
+        load_half(h, x);
         float pm[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) pm[k] = x[k];
 #pragma unroll
-        for (int c = 8; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
-        mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
+        mt = fmaxf(mt, fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))));
       }
       mx = fmaxf(mx, mt);
       const float m_new = fmaxf(m, mt);
@@ -391,17 +411,22 @@ __global__ void __maxnreg__(200)
       const float mref = (m == -INFINITY) ? 0.f : m;
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < BN / 32; ++j) {  // 32 probabilities -> 16 packed columns
-        uint32_t w[16];
+      for (int h = 0; h < NH; ++h) {
+        float x[64];
+        load_half(h, x);  // S columns [64h, 64h+64); P of half h goes to columns [32h, 32h+32)
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float e0 = ex2(x[j * 32 + 2 * c] - mref);
-          const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
-          ps[(2 * c) & 7] += e0;
-          ps[(2 * c + 1) & 7] += e1;
-          w[c] = pack_bf16(e0, e1);
+        for (int j = 0; j < 2; ++j) {
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float e0 = ex2(x[j * 32 + 2 * c] - mref);
+            const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
+            ps[(2 * c) & 7] += e0;
+            ps[(2 * c + 1) & 7] += e1;
+            w[c] = pack_bf16(e0, e1);
+          }
+          tmem_st16(sS + h * 32 + j * 16, w);
         }
-        tmem_st16(sS + j * 16, w);
       }
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       tmem_wait_st();
@@ -456,8 +481,10 @@ static cudaError_t launch2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK, con
                              const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st) {
   using C = Attn2Cfg<D, BN, MODE>;
   auto kern = attn2_kernel<D, BN, MODE>;
-  const int smem = C::SMEM < 116 * 1024 ? 116 * 1024 : C::SMEM;  // one CTA per SM (all 512 TMEM columns)
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  int smem = C::SMEM + (C::kFused ? p.kv_rows_per_head * 4 : 0);  // + FUSED key biases
+  if (smem < 116 * 1024) smem = 116 * 1024;                        // one CTA per SM (all 512 TMEM columns)
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   if (e != cudaSuccess) return e;
   const dim3 grid((p.n_rows + 255) / 256, BH);
   kern<<<grid, C::THREADS, smem, st>>>(tmQ, tmK, tmK2, tmV, p);

@@ -108,7 +108,13 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
   return ISA_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? ISA_OK : ISA_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;  // reported by isa_last_error()
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ISA_OK;
+  g_last_cuda_error = e;
+  return ISA_ERR_CUDA;
+}
 
 // --- tensor maps (driver entry point fetched once through the runtime)
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -467,6 +473,10 @@ int isa_read_device_status(void* ws, void* stream) {
   if (cudaMemsetAsync(at<int>(ws, kStatusOffset), 0, sizeof(int), st) != cudaSuccess) return ISA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return ISA_ERR_CUDA;
   return h;
+}
+
+const char* isa_last_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no CUDA error recorded" : cudaGetErrorString(g_last_cuda_error);
 }
 
 const char* isa_status_string(int status) {
