@@ -374,17 +374,42 @@ __global__ void __launch_bounds__(320, 1)
         }
       };
       float mt = -INFINITY;
+      if constexpr (C::kFused) {
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        float x[64];
-        load_half(h, x);
+        for (int h = 0; h < NH; ++h) {
+          float x[64];
+          load_half(h, x);
+          float pm[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) pm[k] = x[k];
+#pragma unroll
+          for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
+          mt = fmaxf(mt, fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))));
+        }
+      } else {
+        // every S column of the tile in flight at once; max of the raw
+        // scores (the scale is positive), columns past `valid` excluded
+        uint32_t u[BN / 32][32];
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) tmem_ld32(sS + j * 32, u[j]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) regs_after(u[j]);
         float pm[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) pm[k] = x[k];
+        for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
+        if (valid >= BN) {
 #pragma unroll
-        for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
-        mt = fmaxf(mt, fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))));
+          for (int c = 0; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(u[c >> 5][c & 31]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c < valid) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(u[c >> 5][c & 31]));
+        }
+        const float raw = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        mt = raw * p.scale_log2;
       }
       mx = fmaxf(mx, mt);
       const float m_new = fmaxf(m, mt);
@@ -410,22 +435,65 @@ __global__ void __launch_bounds__(320, 1)
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if constexpr (C::kFused) {
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        float x[64];
-        load_half(h, x);  // S columns [64h, 64h+64); P of half h goes to columns [32h, 32h+32)
+        for (int h = 0; h < NH; ++h) {
+          float x[64];
+          load_half(h, x);  // S columns [64h, 64h+64); P of half h goes to columns [32h, 32h+32)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint32_t w[16];
+          for (int j = 0; j < 2; ++j) {
+            uint32_t w[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float e0 = ex2(x[j * 32 + 2 * c] - mref);
-            const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
-            ps[(2 * c) & 7] += e0;
-            ps[(2 * c + 1) & 7] += e1;
-            w[c] = pack_bf16(e0, e1);
+            for (int c = 0; c < 16; ++c) {
+              const float e0 = ex2(x[j * 32 + 2 * c] - mref);
+              const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
+              ps[(2 * c) & 7] += e0;
+              ps[(2 * c + 1) & 7] += e1;
+              w[c] = pack_bf16(e0, e1);
+            }
+            tmem_st16(sS + h * 32 + j * 16, w);
           }
-          tmem_st16(sS + h * 32 + j * 16, w);
+        }
+      } else {
+        // quarters of 32 columns: the next quarter's tcgen05.ld is in flight
+        // while this one is exponentiated; P of quarter q goes to columns
+        // [16q, 16q+16), already consumed (disjoint from the load in flight)
+        const float nm = -mref;
+        uint32_t cur[32];
+        tmem_ld32(sS, cur);
+        tmem_wait_ld();
+#pragma unroll
+        for (int qq = 0; qq < BN / 32; ++qq) {
+          uint32_t nxt[32];
+          if (qq + 1 < BN / 32) tmem_ld32(sS + (qq + 1) * 32, nxt);
+          regs_after(cur);
+          uint32_t w[16];
+          if (valid >= BN) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float e0 = ex2(fmaf(__uint_as_float(cur[2 * c]), p.scale_log2, nm));
+              const float e1 = ex2(fmaf(__uint_as_float(cur[2 * c + 1]), p.scale_log2, nm));
+              ps[(2 * c) & 7] += e0;
+              ps[(2 * c + 1) & 7] += e1;
+              w[c] = pack_bf16(e0, e1);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int col = qq * 32 + 2 * c;
+              const float e0 = col < valid ? ex2(fmaf(__uint_as_float(cur[2 * c]), p.scale_log2, nm)) : 0.f;
+              const float e1 = col + 1 < valid ? ex2(fmaf(__uint_as_float(cur[2 * c + 1]), p.scale_log2, nm)) : 0.f;
+              ps[(2 * c) & 7] += e0;
+              ps[(2 * c + 1) & 7] += e1;
+              w[c] = pack_bf16(e0, e1);
+            }
+          }
+          tmem_st16(sS + qq * 16, w);
+          if (qq + 1 < BN / 32) {
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
+          }
         }
       }
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
