@@ -200,10 +200,16 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--heads", type=int, default=None, help="override H (small profiling captures)")
+    ap.add_argument("--rho", type=float, default=None, help="override rho (profiling captures)")
+    ap.add_argument("--keep", type=float, default=None, help="override keep (profiling captures)")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
     if args.heads:
         cfg = cfg.replace(H=args.heads)
+    if args.rho is not None:
+        cfg = cfg.replace(rho=args.rho)
+    if args.keep is not None:
+        cfg = cfg.replace(keep=args.keep)
     if args.impl == "reference":
         run_reference(args, cfg)
         return

@@ -27,11 +27,13 @@
 // issuer.  TMEM: S/P of tile i at [i*BN, i*BN+BN), O of tile i at
 // [2*BN + i*D, 2*BN + i*D + D).
 //
-// Ordering: S_i(t+1) overwrites the columns that PV_i(t) reads as P_i(t), so
-// the issuer waits for PV_i(t) to complete (o_done[i]) before issuing
-// S_i(t+1); in between it issues PV of the other tile, so the tensor pipe
-// stays fed.  A softmax warpgroup that sees S_i(t) may therefore touch O_i
-// (rescale) and overwrite the S_i columns with P_i(t) without further waits.
+// Ordering: the issuer runs the tensor pipe as PV0(t), S0(t+1), PV1(t),
+// S1(t+1), so each tile's softmax overlaps two MMAs of the other tile.
+// S_i(t+1) overwrites the columns PV_i(t) reads as P_i(t); it is issued
+// behind PV_i(t) by the same thread and UMMAs from one thread execute in
+// order.  The commit that signals S_i(t+1) fires only when every earlier
+// UMMA (PV_i(t) included) is complete, so a softmax warpgroup that sees
+// S_i(t+1) may rescale O_i and overwrite the S_i columns with P_i(t+1).
 // Every mbarrier wait is bounded (status word + CTA abort flag, as in
 // flash.cu).
 #include <cmath>
@@ -256,23 +258,42 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; ok && t < nT; ++t) {
         const int st = t % ST;
         const uint32_t ph = t & 1;
+        const bool more = t + 1 < nT;
         if (!(ok = w1(&bars->v_full[st], (t / ST) & 1, bars, p))) break;
-        if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
-        tc_fence_after();
-        issue_PV(0, t);
-        if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
-        tc_fence_after();
-        issue_PV(1, t);
-        umma_commit(&bars->kv_empty[st]);
-        if (t + 1 < nT) {
-          const int st1 = (t + 1) % ST;
-          if (!(ok = w1(&bars->k_full[st1], ((t + 1) / ST) & 1, bars, p))) break;
-          if (!(ok = w1(&bars->o_done[0], ph, bars, p))) break;
+        if constexpr (ST >= 2) {
+          // Tensor-pipe order PV0(t), S0(t+1), PV1(t), S1(t+1): each softmax
+          // warpgroup has the other tile's PV and S (two MMAs) to hide behind.
+          // S_i(t+1) overwrites the P_i(t) columns that PV_i(t), issued just
+          // before it, reads: UMMAs issued by one thread execute in order.
+          if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
           tc_fence_after();
-          issue_S(0, t + 1);
-          if (!(ok = w1(&bars->o_done[1], ph, bars, p))) break;
+          issue_PV(0, t);
+          if (more) {
+            if (!(ok = w1(&bars->k_full[(t + 1) % ST], ((t + 1) / ST) & 1, bars, p))) break;
+            tc_fence_after();
+            issue_S(0, t + 1);
+          }
+          if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
           tc_fence_after();
-          issue_S(1, t + 1);
+          issue_PV(1, t);
+          umma_commit(&bars->kv_empty[st]);
+          if (more) issue_S(1, t + 1);
+        } else {
+          // One stage: K(t+1) lands only after PV(t) of both tiles released
+          // the stage, so both PVs go first.
+          if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
+          tc_fence_after();
+          issue_PV(0, t);
+          if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
+          tc_fence_after();
+          issue_PV(1, t);
+          umma_commit(&bars->kv_empty[st]);
+          if (more) {
+            if (!(ok = w1(&bars->k_full[0], ((t + 1) / ST) & 1, bars, p))) break;
+            tc_fence_after();
+            issue_S(0, t + 1);
+            issue_S(1, t + 1);
+          }
         }
       }
       umma_commit(&bars->teardown);
