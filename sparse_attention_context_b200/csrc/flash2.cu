@@ -352,10 +352,13 @@ __global__ void __launch_bounds__(320, 1)
     // replaces keeping all BN logits in registers: 10 warps per SM leave
     // 168 registers per thread).
     constexpr int NH = BN / 64;
+    int valid_next = nT > 0 ? kv_count<BN, MODE>(p, bh, 0) : 0;
     for (int t = 0; ok && t < nT; ++t) {
+      const int valid = valid_next;
+      if (t + 1 < nT) valid_next = kv_count<BN, MODE>(p, bh, t + 1);  // prefetched under the wait below
       if (!(ok = wwarp(&bars->s_full[i], t & 1, bars, p))) break;
       tc_fence_after();
-      const int valid = kv_count<BN, MODE>(p, bh, t);
+      uint32_t sreg[C::kFused ? 1 : BN / 32][32];
       const float* bias = C::kFused ? sBias + t * BN : nullptr;
       // logits of half h, in log2 units (-inf outside the tile's tokens)
       auto load_half = [&](int h, float (&x)[64]) {
@@ -410,23 +413,23 @@ __global__ void __launch_bounds__(320, 1)
         }
       } else {
         // every S column of the tile in flight at once; max of the raw
-        // scores (the scale is positive), columns past `valid` excluded
-        uint32_t u[BN / 32][32];
+        // scores (the scale is positive), columns past `valid` excluded.
+        // The scores stay in registers for the exponent pass below.
 #pragma unroll
-        for (int j = 0; j < BN / 32; ++j) tmem_ld32(sS + j * 32, u[j]);
+        for (int j = 0; j < BN / 32; ++j) tmem_ld32(sS + j * 32, sreg[j]);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < BN / 32; ++j) regs_after(u[j]);
+        for (int j = 0; j < BN / 32; ++j) regs_after(sreg[j]);
         float pm[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
         if (valid >= BN) {
 #pragma unroll
-          for (int c = 0; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(u[c >> 5][c & 31]));
+          for (int c = 0; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sreg[c >> 5][c & 31]));
         } else {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
-            if (c < valid) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(u[c >> 5][c & 31]));
+            if (c < valid) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sreg[c >> 5][c & 31]));
         }
         const float raw = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
@@ -437,21 +440,10 @@ __global__ void __launch_bounds__(320, 1)
       // Rescale only when the running maximum grew by more than 2^8: the
       // stale reference keeps every p <= 256, exact after the final 1/l.
       const bool need = m_new > m + 8.0f;
-      if (t > 0 && __any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2(m - m_new) : 1.f;
-#pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
-          uint32_t u[32];
-          tmem_ld32(sO + j * 32, u);
-          tmem_wait_ld();
-          regs_after(u);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
-          tmem_st32(sO + j * 32, u);
-        }
-      }
+      // factor for the accumulated O and l when the reference moves
+      const float alpha = need ? ex2(m - m_new) : 1.f;
       if (need) {
-        l *= ex2(m - m_new);
+        l *= alpha;
         m = m_new;
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
@@ -476,48 +468,49 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       } else {
-        // quarters of 32 columns: the next quarter's tcgen05.ld is in flight
-        // while this one is exponentiated; P of quarter q goes to columns
-        // [16q, 16q+16), already consumed (disjoint from the load in flight)
+        // quarters of 32 columns; P of quarter q goes to columns [16q, 16q+16)
+        // (the scores are already in registers)
         const float nm = -mref;
-        uint32_t cur[32];
-        tmem_ld32(sS, cur);
-        tmem_wait_ld();
 #pragma unroll
         for (int qq = 0; qq < BN / 32; ++qq) {
-          uint32_t nxt[32];
-          if (qq + 1 < BN / 32) tmem_ld32(sS + (qq + 1) * 32, nxt);
-          regs_after(cur);
           uint32_t w[16];
           if (valid >= BN) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-              const float e0 = ex2(fmaf(__uint_as_float(cur[2 * c]), p.scale_log2, nm));
-              const float e1 = ex2(fmaf(__uint_as_float(cur[2 * c + 1]), p.scale_log2, nm));
-              ps[(2 * c) & 7] += e0;
-              ps[(2 * c + 1) & 7] += e1;
+              const float e0 = ex2(fmaf(__uint_as_float(sreg[qq][2 * c]), p.scale_log2, nm));
+              const float e1 = ex2(fmaf(__uint_as_float(sreg[qq][2 * c + 1]), p.scale_log2, nm));
+              ps[c & 7] += e0 + e1;
               w[c] = pack_bf16(e0, e1);
             }
           } else {
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const int col = qq * 32 + 2 * c;
-              const float e0 = col < valid ? ex2(fmaf(__uint_as_float(cur[2 * c]), p.scale_log2, nm)) : 0.f;
-              const float e1 = col + 1 < valid ? ex2(fmaf(__uint_as_float(cur[2 * c + 1]), p.scale_log2, nm)) : 0.f;
-              ps[(2 * c) & 7] += e0;
-              ps[(2 * c + 1) & 7] += e1;
+              const float e0 = col < valid ? ex2(fmaf(__uint_as_float(sreg[qq][2 * c]), p.scale_log2, nm)) : 0.f;
+              const float e1 =
+                  col + 1 < valid ? ex2(fmaf(__uint_as_float(sreg[qq][2 * c + 1]), p.scale_log2, nm)) : 0.f;
+              ps[c & 7] += e0 + e1;
               w[c] = pack_bf16(e0, e1);
             }
           }
           tmem_st16(sS + qq * 16, w);
-          if (qq + 1 < BN / 32) {
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
-          }
         }
       }
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      // O_i rescale (PV_i(t-1) is complete, PV_i(t) not yet issued), done
+      // after the scores left the registers
+      if (t > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          uint32_t u[32];
+          tmem_ld32(sO + j * 32, u);
+          tmem_wait_ld();
+          regs_after(u);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+          tmem_st32(sO + j * 32, u);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[i]);
