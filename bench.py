@@ -296,7 +296,7 @@ def main():
     # in-house dense kernel on the same inputs (the baseline the metric names)
     dense_ms = None
     if not args.no_dense:
-        dws = api.dense_workspace(dev)
+        dws = api.dense_workspace(cfg.d, dev)
         dout = torch.empty_like(q)
         nd = max(2, min(args.steps, 5))
         for _ in range(2):

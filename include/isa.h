@@ -145,9 +145,11 @@ int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, co
 
 /* In-house dense flash attention (the latency baseline; equals ISA at
  * keep = rho = 1): out = softmax(scale q k^T) v over all N keys, per (b, h),
- * non-causal.  scale <= 0 selects 1/sqrt(d).  ws is a control block of at
- * least isa_dense_workspace_size() bytes (status word as above). */
-size_t isa_dense_workspace_size(void);
+ * non-causal.  scale <= 0 selects 1/sqrt(d).  ws: a zeroed buffer of
+ * isa_dense_workspace_size(d) bytes (control block as above, then scratch
+ * for the key-split tail; a smaller ws >= 256 bytes also works, without
+ * the split).  isa_dense_workspace_size returns 0 for an unsupported d. */
+size_t isa_dense_workspace_size(int d);
 int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* q,
                        const uint16_t* k, const uint16_t* v, uint16_t* out,
                        void* ws, size_t ws_bytes, void* stream);

@@ -170,8 +170,11 @@ def isa_forward(q, k, v, N_src: int, block: int, keep: float, rho: float, scale:
     return o
 
 
-def dense_workspace(device="cuda") -> torch.Tensor:
-    return torch.zeros(lib().isa_dense_workspace_size(), dtype=torch.uint8, device=device)
+def dense_workspace(d: int = 128, device="cuda") -> torch.Tensor:
+    n = lib().isa_dense_workspace_size(int(d))
+    if n == 0:
+        raise ValueError("unsupported head dimension")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def isa_dense_attn_fwd(q, k, v, scale: float = 0.0, out=None, ws=None, stream=None):
@@ -179,9 +182,9 @@ def isa_dense_attn_fwd(q, k, v, scale: float = 0.0, out=None, ws=None, stream=No
     if out is None:
         out = torch.empty_like(q)
     _check_qkv(q, k, v, out)
-    if ws is None:
-        ws = dense_workspace(q.device)
     B, H, N, d = q.shape
+    if ws is None:
+        ws = dense_workspace(d, q.device)
     rc = lib().isa_dense_attn_fwd(B, H, N, d, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                   out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
     check("isa_dense_attn_fwd", rc)

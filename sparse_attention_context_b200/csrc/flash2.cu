@@ -22,6 +22,10 @@
 //          the Taylor output of every row (routed rows are overwritten by
 //          the FULL pass afterwards).
 //
+// Work items: 256 query rows of one (b, h); whole waves of items run as
+// one launch, the items of a partial last wave are split along the key
+// tiles over all SMs and merged by combine_kernel (no idle tail wave).
+//
 // Warps (320 threads): 0-3 softmax of tile 0, 4-7 softmax of tile 1 (thread
 // <-> query row <-> TMEM lane), 8 TMA producer, 9 TMEM allocator + UMMA
 // issuer.  TMEM: S/P of tile i at [i*BN, i*BN+BN), O of tile i at
@@ -136,9 +140,15 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t aKV = smem_u32(smem + C::OFF_KV);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.y;
-  const int row0 = blockIdx.x * 256;
-  const int nT = p.n_kv_tiles;
+  const bool split = p.split_pieces > 0;
+  const int item = p.item_base + (split ? static_cast<int>(blockIdx.x) / p.split_pieces : static_cast<int>(blockIdx.x));
+  const int piece = split ? static_cast<int>(blockIdx.x) % p.split_pieces : 0;
+  const int pieces = split ? p.split_pieces : 1;
+  const int bh = item / p.pairs_per_head;
+  const int row0 = (item % p.pairs_per_head) * 256;
+  // key tiles [kv0, kv0 + nT) of this CTA (all of them unless key-split)
+  const int kv0 = piece * p.n_kv_tiles / pieces;
+  const int nT = (piece + 1) * p.n_kv_tiles / pieces - kv0;
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -187,7 +197,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < nT; ++t) {
         const int st = t % ST;
         if (t >= ST && !w1(&bars->kv_empty[st], ((t / ST) - 1) & 1, bars, p)) break;
-        const int r = kv_row<BN, MODE>(p, bh, t);
+        const int r = kv_row<BN, MODE>(p, bh, kv0 + t);
         uint8_t* base = smem + C::OFF_KV + st * C::STAGE_BYTES;
         mbar_arrive_expect_tx(&bars->k_full[st], (C::kFused ? 2 : 1) * C::KT_BYTES);
 #pragma unroll
@@ -352,14 +362,14 @@ __global__ void __launch_bounds__(320, 1)
     // replaces keeping all BN logits in registers: 10 warps per SM leave
     // 168 registers per thread).
     constexpr int NH = BN / 64;
-    int valid_next = nT > 0 ? kv_count<BN, MODE>(p, bh, 0) : 0;
+    int valid_next = nT > 0 ? kv_count<BN, MODE>(p, bh, kv0) : 0;
     for (int t = 0; ok && t < nT; ++t) {
       const int valid = valid_next;
-      if (t + 1 < nT) valid_next = kv_count<BN, MODE>(p, bh, t + 1);  // prefetched under the wait below
+      if (t + 1 < nT) valid_next = kv_count<BN, MODE>(p, bh, kv0 + t + 1);  // prefetched under the wait below
       if (!(ok = wwarp(&bars->s_full[i], t & 1, bars, p))) break;
       tc_fence_after();
       uint32_t sreg[C::kFused ? 1 : BN / 32][32];
-      const float* bias = C::kFused ? sBias + t * BN : nullptr;
+      const float* bias = C::kFused ? sBias + (kv0 + t) * BN : nullptr;
       // logits of half h, in log2 units (-inf outside the tile's tokens)
       auto load_half = [&](int h, float (&x)[64]) {
         if constexpr (C::kFused) {
@@ -526,6 +536,23 @@ __global__ void __launch_bounds__(320, 1)
         // sharpness = max_b softmax_b = 2^(mx - m) / l (l is relative to m)
         if (store) p.sharp[static_cast<size_t>(bh) * p.N + dst] = ex2(mx - m) / l;
       }
+      if (split) {
+        // unnormalised partial accumulator of this key range (+ its m, l)
+        const size_t prow = static_cast<size_t>(blockIdx.x) * 256 + i * 128 + r;
+        p.ml_part[prow] = make_float2(m, l);
+        float4* op = reinterpret_cast<float4*>(p.o_part + prow * D);
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          uint32_t u[32];
+          tmem_ld32(sO + j * 32, u);
+          tmem_wait_ld();
+          regs_after(u);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            op[j * 8 + q4] = make_float4(__uint_as_float(u[4 * q4]), __uint_as_float(u[4 * q4 + 1]),
+                                         __uint_as_float(u[4 * q4 + 2]), __uint_as_float(u[4 * q4 + 3]));
+        }
+      } else {
       uint16_t* orow = p.out + (static_cast<size_t>(bh) * p.N + dst) * D;
       const float inv = 1.f / l;
 #pragma unroll
@@ -547,6 +574,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
+      }
     }
   }
 
@@ -558,19 +586,93 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
+// Merge of key-split partials: row r of split item s is
+// sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p with M = max_p m_p.
+// One warp per query row; grid covers n_items * 256 rows.
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o_part,
+                                                      const float2* __restrict__ ml_part, int pieces, int item_base,
+                                                      int n_items, const FlashParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rr_all = blockIdx.x * 8 + warp;
+  if (rr_all >= n_items * 256) return;
+  const int s = rr_all / 256, rr = rr_all % 256;
+  const int item = item_base + s;
+  const int bh = item / p.pairs_per_head;
+  const int g = (item % p.pairs_per_head) * 256 + rr;
+  if (g >= p.n_rows) return;
+  int dst = p.row_idx ? __ldg(p.row_idx + static_cast<size_t>(bh) * p.n_rows + g) : g;
+  if (static_cast<unsigned>(dst) >= static_cast<unsigned>(p.N)) {
+    if (lane == 0 && p.status != nullptr) atomicCAS(p.status, 0, 1);
+    return;
+  }
+  float M = -INFINITY;
+  for (int q = 0; q < pieces; ++q) M = fmaxf(M, ml_part[(static_cast<size_t>(s) * pieces + q) * 256 + rr].x);
+  constexpr int CPL = D / 32;  // columns per lane
+  float acc[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+  float L = 0.f;
+  for (int q = 0; q < pieces; ++q) {
+    const size_t prow = (static_cast<size_t>(s) * pieces + q) * 256 + rr;
+    const float2 ml = ml_part[prow];
+    const float w = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
+    L += w * ml.y;
+    const float* op = o_part + prow * D + lane * CPL;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[c] = fmaf(w, op[c], acc[c]);
+  }
+  const float inv = 1.f / L;
+  uint16_t* orow = p.out + (static_cast<size_t>(bh) * p.N + dst) * D + lane * CPL;
+#pragma unroll
+  for (int c = 0; c < CPL; c += 2) *reinterpret_cast<uint32_t*>(orow + c) = pack_bf16(acc[c] * inv, acc[c + 1] * inv);
+}
+
 template <int D, int BN, int MODE>
 static cudaError_t launch2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmK2,
-                             const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st) {
+                             const CUtensorMap& tmV, const FlashParams& p0, int BH, cudaStream_t st) {
   using C = Attn2Cfg<D, BN, MODE>;
   auto kern = attn2_kernel<D, BN, MODE>;
-  int smem = C::SMEM + (C::kFused ? p.kv_rows_per_head * 4 : 0);  // + FUSED key biases
-  if (smem < 116 * 1024) smem = 116 * 1024;                        // one CTA per SM (all 512 TMEM columns)
+  int smem = C::SMEM + (C::kFused ? p0.kv_rows_per_head * 4 : 0);  // + FUSED key biases
+  if (smem < 116 * 1024) smem = 116 * 1024;                         // one CTA per SM (all 512 TMEM columns)
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   if (e != cudaSuccess) return e;
-  const dim3 grid((p.n_rows + 255) / 256, BH);
-  kern<<<grid, C::THREADS, smem, st>>>(tmQ, tmK, tmK2, tmV, p);
-  return cudaGetLastError();
+  FlashParams p = p0;
+  p.pairs_per_head = (p.n_rows + 255) / 256;
+  p.item_base = 0;
+  p.split_pieces = 0;
+  const long long items = static_cast<long long>(BH) * p.pairs_per_head;
+  // Whole waves as they are; the remainder split along the keys over the SMs
+  // (one CTA per SM), then merged, so that no SM idles through a last wave.
+  int dev = 0, nsm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long long whole = nsm > 0 ? items / nsm * nsm : items;
+  const int rem = static_cast<int>(items - whole);
+  int pieces = 0;
+  if (!C::kFused && rem > 0 && p.o_part != nullptr && p.split_capacity > 0) {
+    pieces = nsm / rem;
+    if (pieces > p.n_kv_tiles / 4) pieces = p.n_kv_tiles / 4;
+    while (pieces > 1 && pieces * rem > p.split_capacity) --pieces;
+    if (pieces < 2) pieces = 0;
+  }
+  const long long first = pieces ? whole : items;
+  if (first > 0) {
+    kern<<<static_cast<unsigned>(first), C::THREADS, smem, st>>>(tmQ, tmK, tmK2, tmV, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (pieces) {
+    FlashParams ps = p;
+    ps.item_base = static_cast<int>(whole);
+    ps.split_pieces = pieces;
+    kern<<<static_cast<unsigned>(rem * pieces), C::THREADS, smem, st>>>(tmQ, tmK, tmK2, tmV, ps);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    combine_kernel<D><<<(rem * 256 + 7) / 8, 256, 0, st>>>(p.o_part, p.ml_part, pieces, static_cast<int>(whole), rem,
+                                                           p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,

@@ -21,8 +21,21 @@ struct Dims {
 };
 
 struct WsLayout {
-  size_t Qbar, Kbar, Vbar, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, total;
+  size_t Qbar, Kbar, Vbar, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, opart, mlpart, total;
+  int split_ctas;  // key-split partial CTAs the workspace holds
 };
+
+// SMs of the current device (the key-split partial buffers hold one CTA per
+// SM); 148 when no device is visible (sizing on a host without a GPU).
+int split_ctas_for_device() {
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) !=
+                                               cudaSuccess || nsm <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return nsm;
+}
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -91,6 +104,9 @@ WsLayout layout(const Dims& d) {
   L.kept = take(BH * std::max(d.n_keep, 1) * 4);
   L.routed = take(BH * std::max(d.n_route, 1) * 4);
   L.taylor = take(BH * std::max(d.N - d.n_route, 1) * 4);
+  L.split_ctas = split_ctas_for_device();
+  L.opart = take(static_cast<size_t>(L.split_ctas) * 256 * d.d * 4);
+  L.mlpart = take(static_cast<size_t>(L.split_ctas) * 256 * 8);
   L.total = off;
   return L;
 }
@@ -146,6 +162,9 @@ struct Ctx {
 
 FlashParams base_params(const Ctx& c) {
   FlashParams p{};
+  p.o_part = at<float>(c.ws, c.L.opart);
+  p.ml_part = at<float2>(c.ws, c.L.mlpart);
+  p.split_capacity = c.L.split_ctas;
   p.N = c.d.N;
   p.N_src = c.d.N_src;
   p.N_ctx = c.d.N_ctx;
@@ -432,7 +451,11 @@ int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, co
   return rc;
 }
 
-size_t isa_dense_workspace_size(void) { return kCtlBytes; }
+size_t isa_dense_workspace_size(int d) {
+  if (d != 64 && d != 128) return 0;
+  const int nsm = split_ctas_for_device();
+  return kCtlBytes + 4096 + align256(static_cast<size_t>(nsm) * 256 * d * 4) + align256(static_cast<size_t>(nsm) * 256 * 8);
+}
 
 int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* q, const uint16_t* k,
                        const uint16_t* v, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
@@ -443,6 +466,9 @@ int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* 
   if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
   int rc = check_ws(ws, ws_bytes, kCtlBytes);
   if (rc != ISA_OK) return rc;
+  // key-split partials after the control block, as many CTAs as fit
+  const size_t per = split_bytes_per_cta(d);
+  const int cap = ws_bytes > kCtlBytes + 4096 ? static_cast<int>((ws_bytes - kCtlBytes - 4096) / per) : 0;
   CUtensorMap tmQ, tmK, tmV;
   if (!make_tmap_bf16(&tmQ, q, static_cast<uint64_t>(BH) * N, d, 128) ||
       !make_tmap_bf16(&tmK, k, static_cast<uint64_t>(BH) * N, d, 128) ||
@@ -459,6 +485,11 @@ int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* 
   p.scale_log2 = (scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d))) * 1.4426950408889634f;
   p.status = at<int>(ws, kStatusOffset);
   p.inject = at<int>(ws, kInjectOffset);
+  if (cap > 0) {
+    p.o_part = at<float>(ws, kCtlBytes);
+    p.ml_part = at<float2>(ws, align256(kCtlBytes + static_cast<size_t>(cap) * 256 * d * 4));
+    p.split_capacity = cap;
+  }
   return cuda_status(launch_attn2(d, 128, MODE_DENSE, tmQ, tmK, tmK, tmV, p, static_cast<int>(BH),
                                   static_cast<cudaStream_t>(stream)));
 }

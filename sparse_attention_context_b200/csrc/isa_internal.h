@@ -36,7 +36,21 @@ struct FlashParams {
   float scale_log2;       // s * log2(e)
   int* status;            // device status word or null
   const int* inject;      // device fault-injection word or null
+  // two-tile engine only: work items are (b*H + h) * pairs_per_head + pair
+  // (256 query rows each); a launch covers items from item_base.
+  int item_base;
+  int pairs_per_head;
+  // key-split launch (split_pieces > 0): CTA g handles item
+  // item_base + g / split_pieces over key tiles [piece*nT/pieces,
+  // (piece+1)*nT/pieces) and writes unnormalised partials instead of out.
+  int split_pieces;
+  float* o_part;          // [CTAs, 256, D] fp32 partial accumulators
+  float2* ml_part;        // [CTAs, 256] (reference max in log2 units, sum)
+  int split_capacity;     // CTAs the partial buffers hold (0 = no split)
 };
+
+// Bytes per CTA of key-split partials for head dim D.
+inline size_t split_bytes_per_cta(int D) { return 256ull * (static_cast<size_t>(D) * 4 + 8); }
 
 // Tensor map over a [rows, D] bf16 row-major matrix, box = 64 columns x
 // box_rows rows, 128-byte swizzle.  Returns false if encoding fails.

@@ -65,7 +65,8 @@ def test_workspace_size(L):
     assert n >= 3 * BH * nB * d * 4 + BH * N * 4 + BH * N * 4
     assert n < 64 * 2**20
     assert L.isa_workspace_size(ctypes.byref(shape(d=96))) == 0
-    assert L.isa_dense_workspace_size() >= 8
+    assert L.isa_dense_workspace_size(128) >= 256 + 148 * 256 * 128 * 4
+    assert L.isa_dense_workspace_size(96) == 0
 
 
 @pytest.mark.parametrize("bad,code", [

@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 def test_dense_matches_oracle(cuda_ok, d, N_src, N_ctx, H):
     cfg = CONFIGS["tiny"].replace(H=H, d=d, N_src=N_src, N_ctx=N_ctx)
     bits, (q, k, v) = inputs(cfg)
-    ws = api.dense_workspace()
+    ws = api.dense_workspace(q.shape[-1])
     out = api.isa_dense_attn_fwd(q, k, v, ws=ws)
     assert api.isa_read_device_status(ws) == 0
     o = bf16_bits_to_f64(from_torch_bf16(out))

@@ -33,7 +33,7 @@ def test_injected_timeout_is_reported_and_recovered(cuda_ok):
 def test_injected_timeout_dense(cuda_ok):
     cfg = CONFIGS["tiny"]
     _, (q, k, v) = inputs(cfg)
-    ws = api.dense_workspace()
+    ws = api.dense_workspace(q.shape[-1])
     ws[4:8].view(torch.int32).fill_(1)
     api.isa_dense_attn_fwd(q, k, v, ws=ws)
     assert api.isa_read_device_status(ws) == 5
