@@ -74,6 +74,7 @@ struct Attn2Bars {
   uint64_t v_full[3];
   uint64_t kv_empty[3];
   uint64_t s_full[2];
+  uint64_t p_full[2];  // all 128 threads of a tile wrote P (and rescaled O)
   uint64_t o_done[2];
   uint64_t teardown[2];
   uint32_t tmem_base;
@@ -89,27 +90,16 @@ __device__ __forceinline__ bool w1(uint64_t* bar, uint32_t par, Attn2Bars* bars,
   if (r == 2) raise2(bars, p);
   return r == 0;
 }
+// Bounded busy wait of the issuing thread (reacts at once when the phase completes).
+__device__ __forceinline__ bool wspin(uint64_t* bar, uint32_t par, Attn2Bars* bars, const FlashParams& p) {
+  const int r = mbar_spin_bounded(bar, par, reinterpret_cast<volatile int*>(&bars->abort), kWaitLimitNs);
+  if (r == 2) raise2(bars, p);
+  return r == 0;
+}
 __device__ __forceinline__ bool wwarp(uint64_t* bar, uint32_t par, Attn2Bars* bars, const FlashParams& p) {
   const bool ok = w1(bar, par, bars, p);
   return __all_sync(0xffffffffu, ok);
 }
-// Barrier of the 128 threads of one softmax warpgroup (named barrier `id`)
-// that also ANDs a predicate across them, so every thread leaves with the
-// same verdict.  All 128 threads reach it every iteration (nothing breaks
-// out of the loop before it), so it cannot wait forever.
-__device__ __forceinline__ bool wg_vote_and(int id, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, %2, 128, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}\n"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id)
-      : "memory");
-  return r != 0;
-}
-
 template <int N>
 __device__ __forceinline__ void regs_after(uint32_t (&r)[N]) {
 #pragma unroll
@@ -168,8 +158,9 @@ __global__ void __launch_bounds__(320, 1)
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->q_full[i], 1);
+      mbar_init(&bars->q_full[i], C::kTmaQ ? 1 : 128);
       mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
       mbar_init(&bars->o_done[i], 1);
       mbar_init(&bars->teardown[i], 1);
     }
@@ -301,6 +292,7 @@ __global__ void __launch_bounds__(320, 1)
                      vals[it].z, vals[it].w);
       }
       fence_proxy_async_smem();
+      mbar_arrive(&bars->q_full[i]);
     }
 
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -321,16 +313,15 @@ __global__ void __launch_bounds__(320, 1)
     }
     // Thread 0 of the warpgroup issues every UMMA of this tile.
     const bool issuer = r == 0;
-    ok = wg_vote_and(2 + i, ok);  // Q rows written by this warpgroup are complete (FULL)
     if (issuer && ok && nT > 0) {
-      bool e = true;
-      if constexpr (C::kTmaQ) e = w1(&bars->q_full[i], 0, bars, p);
+      bool e = w1(&bars->q_full[i], 0, bars, p);  // TMA rows, or this warpgroup's gathered rows
       if (e) e = w1(&bars->k_full[0], 0, bars, p);
       if (e) {
         tc_fence_after();
         issue_S(i, 0);
       }
     }
+    __syncwarp();  // the issuer's warp-mates block here instead of spinning beside it
     // Softmax on 64-column halves of the S tile (a second tcgen05.ld of S
     // replaces keeping all BN logits in registers: 10 warps per SM leave
     // 168 registers per thread).
@@ -339,8 +330,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int t = 0; ok && t < nT; ++t) {
       const int valid = valid_next;
       if (t + 1 < nT) valid_next = kv_count<BN, MODE>(p, bh, kv0 + t + 1);  // prefetched under the wait below
-      const bool okw = wwarp(&bars->s_full[i], t & 1, bars, p);
-      if (okw) {
+      if (!(ok = wwarp(&bars->s_full[i], t & 1, bars, p))) break;
+      {
       tc_fence_after();
       uint32_t sreg[C::kFused ? 1 : BN / 32][32];
       const float* bias = C::kFused ? sBias + (kv0 + t) * BN : nullptr;
@@ -500,12 +491,13 @@ __global__ void __launch_bounds__(320, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      }  // okw
-      // P_i(t) and the O_i rescale are in TMEM for all 128 rows: the issuer
-      // runs PV_i(t), then S_i(t+1) into the same columns (in order).
-      ok = wg_vote_and(2 + i, okw);
-      if (!ok) break;
-      if (issuer) {
+      }
+      mbar_arrive(&bars->p_full[i]);
+      // Once all 128 rows of P_i(t) (and the O_i rescale) are in TMEM, the
+      // issuer runs PV_i(t), then S_i(t+1) into the same columns (in order).
+      // Every wait is a bounded mbarrier wait; failures raise the CTA abort
+      // flag, which ends the other threads' waits.
+      if (issuer && wspin(&bars->p_full[i], t & 1, bars, p)) {
         tc_fence_after();
         const int st = t % ST;
         if (w1(&bars->v_full[st], (t / ST) & 1, bars, p)) {
@@ -513,6 +505,7 @@ __global__ void __launch_bounds__(320, 1)
           if (t + 1 < nT && w1(&bars->k_full[(t + 1) % ST], ((t + 1) / ST) & 1, bars, p)) issue_S(i, t + 1);
         }
       }
+      __syncwarp();  // S_i(t+1) is issued before this warp waits for it
     }
 
     const bool valid_row = g < p.n_rows;

@@ -44,6 +44,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of a phase (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded busy wait (test_wait, never suspends): for a single thread that
+// must react at once.  Returns 0 on success, 1 on abort, 2 on timeout.
+__device__ __forceinline__ int mbar_spin_bounded(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                                 uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return 0;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_test_wait(bar, parity)) return 0;
+    if (abort != nullptr && *abort) return 1;
+    if (global_timer_ns() - t0 > limit_ns) return 2;
+  }
+}
+
 // Bounded wait for the phase with the given parity to complete.
 // Returns 0 on success, 1 when *abort became non-zero, 2 on timeout.
 __device__ __forceinline__ int mbar_wait_bounded(uint64_t* bar, uint32_t parity, const volatile int* abort,
