@@ -74,9 +74,9 @@ struct Attn2Bars {
   uint64_t v_full[3];
   uint64_t kv_empty[3];
   uint64_t s_full[2];
-  uint64_t p_full[2];  // all 128 threads of a tile wrote P (and rescaled O)
+  uint64_t p_full[2];
   uint64_t o_done[2];
-  uint64_t teardown[2];
+  uint64_t teardown;
   uint32_t tmem_base;
   int abort;
 };
@@ -87,12 +87,6 @@ __device__ __forceinline__ void raise2(Attn2Bars* bars, const FlashParams& p) {
 }
 __device__ __forceinline__ bool w1(uint64_t* bar, uint32_t par, Attn2Bars* bars, const FlashParams& p) {
   const int r = mbar_wait_bounded(bar, par, reinterpret_cast<volatile int*>(&bars->abort), kWaitLimitNs);
-  if (r == 2) raise2(bars, p);
-  return r == 0;
-}
-// Bounded busy wait of the issuing thread (reacts at once when the phase completes).
-__device__ __forceinline__ bool wspin(uint64_t* bar, uint32_t par, Attn2Bars* bars, const FlashParams& p) {
-  const int r = mbar_spin_bounded(bar, par, reinterpret_cast<volatile int*>(&bars->abort), kWaitLimitNs);
   if (r == 2) raise2(bars, p);
   return r == 0;
 }
@@ -162,13 +156,13 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->p_full[i], 128);
       mbar_init(&bars->o_done[i], 1);
-      mbar_init(&bars->teardown[i], 1);
     }
     for (int s = 0; s < 3; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 2);  // one commit per tile after its PV
+      mbar_init(&bars->kv_empty[s], 1);
     }
+    mbar_init(&bars->teardown, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -186,38 +180,6 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-
-  // UMMA groups, issued by one elected thread per tile (the UMMAs of a tile
-  // come from a single thread, so they execute in issue order).
-  constexpr uint32_t IDS = idesc_bf16(128, BN, 0);
-  constexpr uint32_t IDO = idesc_bf16(128, D, 1);
-  auto issue_S = [&](int i, int t) {  // S_i = Q_i K_t^T (+ Q_i Klo_t^T), then signal s_full[i]
-    const int st = t % ST;
-    const uint32_t kb = aKV + st * C::STAGE_BYTES;
-    const uint32_t qa = aQ + i * C::Q_BYTES;
-    const uint32_t dS = tmem + i * BN;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk)
-      umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
-                desc_k_sw128(kb + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, kk > 0 ? 1u : 0u);
-    if constexpr (C::kFused) {
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
-                  desc_k_sw128(kb + C::KT_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, 1u);
-    }
-    umma_commit(&bars->s_full[i]);
-  };
-  auto issue_PV = [&](int i, int t) {  // O_i += P_i V_t (P_i from TMEM), then signal o_done[i], kv_empty
-    const int st = t % ST;
-    const uint32_t vb = aKV + st * C::STAGE_BYTES + (C::NKT - 1) * C::KT_BYTES;
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk)
-      umma_bf16_tmem_a(tmem + 2 * BN + i * D, tmem + i * BN + kk * 8, desc_mn_sw128(vb + kk * 16 * 128, BN * 128),
-                       IDO, (t > 0 || kk > 0) ? 1u : 0u);
-    umma_commit(&bars->o_done[i]);
-    umma_commit(&bars->kv_empty[st]);
-  };
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -261,6 +223,91 @@ __global__ void __launch_bounds__(320, 1)
         mbar_wait_bounded(&bars->q_full[0], 0, nullptr, kWaitLimitNs);
         mbar_wait_bounded(&bars->q_full[1], 0, nullptr, kWaitLimitNs);
       }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDS = idesc_bf16(128, BN, 0);
+      constexpr uint32_t IDO = idesc_bf16(128, D, 1);
+      bool ok = w1(&bars->q_full[0], 0, bars, p) && w1(&bars->q_full[1], 0, bars, p);
+      tc_fence_after();
+      auto issue_S = [&](int i, int t) {
+        const int st = t % ST;
+        const uint32_t kb = aKV + st * C::STAGE_BYTES;
+        const uint32_t qa = aQ + i * C::Q_BYTES;
+        const uint32_t dS = tmem + i * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                    desc_k_sw128(kb + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, kk > 0 ? 1u : 0u);
+        if constexpr (C::kFused) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                      desc_k_sw128(kb + C::KT_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, 1u);
+        }
+        umma_commit(&bars->s_full[i]);
+      };
+      auto issue_PV = [&](int i, int t) {
+        const int st = t % ST;
+        const uint32_t vb = aKV + st * C::STAGE_BYTES + (C::NKT - 1) * C::KT_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_tmem_a(tmem + 2 * BN + i * D, tmem + i * BN + kk * 8, desc_mn_sw128(vb + kk * 16 * 128, BN * 128),
+                           IDO, (t > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bars->o_done[i]);
+      };
+      if (ok && nT > 0) {
+        ok = w1(&bars->k_full[0], 0, bars, p);
+        if (ok) {
+          tc_fence_after();
+          issue_S(0, 0);
+          issue_S(1, 0);
+        }
+      }
+      for (int t = 0; ok && t < nT; ++t) {
+        const int st = t % ST;
+        const uint32_t ph = t & 1;
+        const bool more = t + 1 < nT;
+        if (!(ok = w1(&bars->v_full[st], (t / ST) & 1, bars, p))) break;
+        if constexpr (ST >= 2) {
+          // Tensor-pipe order PV0(t), S0(t+1), PV1(t), S1(t+1): each softmax
+          // warpgroup has the other tile's PV and S (two MMAs) to hide behind.
+          // S_i(t+1) overwrites the P_i(t) columns that PV_i(t), issued just
+          // before it, reads: UMMAs issued by one thread execute in order.
+          if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
+          tc_fence_after();
+          issue_PV(0, t);
+          if (more) {
+            if (!(ok = w1(&bars->k_full[(t + 1) % ST], ((t + 1) / ST) & 1, bars, p))) break;
+            tc_fence_after();
+            issue_S(0, t + 1);
+          }
+          if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
+          tc_fence_after();
+          issue_PV(1, t);
+          umma_commit(&bars->kv_empty[st]);
+          if (more) issue_S(1, t + 1);
+        } else {
+          // One stage: K(t+1) lands only after PV(t) of both tiles released
+          // the stage, so both PVs go first.
+          if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
+          tc_fence_after();
+          issue_PV(0, t);
+          if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
+          tc_fence_after();
+          issue_PV(1, t);
+          umma_commit(&bars->kv_empty[st]);
+          if (more) {
+            if (!(ok = w1(&bars->k_full[0], ((t + 1) / ST) & 1, bars, p))) break;
+            tc_fence_after();
+            issue_S(0, t + 1);
+            issue_S(1, t + 1);
+          }
+        }
+      }
+      umma_commit(&bars->teardown);
+      mbar_wait_bounded(&bars->teardown, 0, nullptr, kWaitLimitNs);
     }
   } else {
     // ------------------------------------------ softmax warpgroup of tile i
@@ -311,17 +358,6 @@ __global__ void __launch_bounds__(320, 1)
         sBias[c] = __ldg(p.bias2 + static_cast<size_t>(bh) * p.kv_rows_per_head + c);
       asm volatile("bar.sync 1, 256;" ::: "memory");  // the two softmax warpgroups only
     }
-    // Thread 0 of the warpgroup issues every UMMA of this tile.
-    const bool issuer = r == 0;
-    if (issuer && ok && nT > 0) {
-      bool e = w1(&bars->q_full[i], 0, bars, p);  // TMA rows, or this warpgroup's gathered rows
-      if (e) e = w1(&bars->k_full[0], 0, bars, p);
-      if (e) {
-        tc_fence_after();
-        issue_S(i, 0);
-      }
-    }
-    __syncwarp();  // the issuer's warp-mates block here instead of spinning beside it
     // Softmax on 64-column halves of the S tile (a second tcgen05.ld of S
     // replaces keeping all BN logits in registers: 10 warps per SM leave
     // 168 registers per thread).
@@ -331,7 +367,6 @@ __global__ void __launch_bounds__(320, 1)
       const int valid = valid_next;
       if (t + 1 < nT) valid_next = kv_count<BN, MODE>(p, bh, kv0 + t + 1);  // prefetched under the wait below
       if (!(ok = wwarp(&bars->s_full[i], t & 1, bars, p))) break;
-      {
       tc_fence_after();
       uint32_t sreg[C::kFused ? 1 : BN / 32][32];
       const float* bias = C::kFused ? sBias + (kv0 + t) * BN : nullptr;
@@ -491,21 +526,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      }
       mbar_arrive(&bars->p_full[i]);
-      // Once all 128 rows of P_i(t) (and the O_i rescale) are in TMEM, the
-      // issuer runs PV_i(t), then S_i(t+1) into the same columns (in order).
-      // Every wait is a bounded mbarrier wait; failures raise the CTA abort
-      // flag, which ends the other threads' waits.
-      if (issuer && wspin(&bars->p_full[i], t & 1, bars, p)) {
-        tc_fence_after();
-        const int st = t % ST;
-        if (w1(&bars->v_full[st], (t / ST) & 1, bars, p)) {
-          issue_PV(i, t);
-          if (t + 1 < nT && w1(&bars->k_full[(t + 1) % ST], ((t + 1) / ST) & 1, bars, p)) issue_S(i, t + 1);
-        }
-      }
-      __syncwarp();  // S_i(t+1) is issued before this warp waits for it
     }
 
     const bool valid_row = g < p.n_rows;
@@ -560,10 +581,6 @@ __global__ void __launch_bounds__(320, 1)
     }
   }
 
-  if (warp < 8 && (tid & 127) == 0) {  // every UMMA this tile's issuer started is done
-    umma_commit(&bars->teardown[warp >> 2]);
-    mbar_wait_bounded(&bars->teardown[warp >> 2], 0, nullptr, kWaitLimitNs);
-  }
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
