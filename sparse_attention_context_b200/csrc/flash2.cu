@@ -433,9 +433,11 @@ __global__ void __launch_bounds__(320, 1)
         float pm[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
-        if (valid >= BN) {
+        if (valid >= BN) {  // three-input max: 64 instructions for 128 scores
 #pragma unroll
-          for (int c = 0; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sreg[c >> 5][c & 31]));
+          for (int c = 0; c < BN; c += 2)
+            pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], __uint_as_float(sreg[c >> 5][c & 31]),
+                                     __uint_as_float(sreg[c >> 5][(c + 1) & 31]));
         } else {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
@@ -458,6 +460,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       if constexpr (C::kFused) {
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
@@ -472,7 +475,7 @@ __global__ void __launch_bounds__(320, 1)
               const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
               ps[(2 * c) & 7] += e0;
               ps[(2 * c + 1) & 7] += e1;
-              w[c] = pack_bf16_pos(e0, e1);
+              w[c] = pack_bf16(e0, e1);
             }
             tmem_st16(sS + h * 32 + j * 16, w);
           }
@@ -481,19 +484,20 @@ __global__ void __launch_bounds__(320, 1)
         // quarters of 32 columns; P of quarter q goes to columns [16q, 16q+16)
         // (the scores are already in registers)
         const float nm = -mref;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(nm, nm);
 #pragma unroll
         for (int qq = 0; qq < BN / 32; ++qq) {
           uint32_t w[16];
           if (valid >= BN) {
+            // packed fp32x2 FMA (argument) and add (row sum): half the instructions
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-              // a quarter of the exponentials on the FMA pipe, the rest on MUFU
-              const float a0 = fmaf(__uint_as_float(sreg[qq][2 * c]), p.scale_log2, nm);
-              const float a1 = fmaf(__uint_as_float(sreg[qq][2 * c + 1]), p.scale_log2, nm);
-              const float e0 = (c & 3) == 3 ? ex2_poly(a0) : ex2(a0);
-              const float e1 = (c & 3) == 3 ? ex2_poly(a1) : ex2(a1);
-              ps[c & 7] += e0 + e1;
-              w[c] = pack_bf16_pos(e0, e1);
+              const float2 a = __ffma2_rn(
+                  make_float2(__uint_as_float(sreg[qq][2 * c]), __uint_as_float(sreg[qq][2 * c + 1])), sc2, nm2);
+              const float e0 = ex2(a.x);
+              const float e1 = ex2(a.y);
+              ps2[c & 3] = __fadd2_rn(ps2[c & 3], make_float2(e0, e1));
+              w[c] = pack_bf16(e0, e1);
             }
           } else {
 #pragma unroll
@@ -503,11 +507,15 @@ __global__ void __launch_bounds__(320, 1)
               const float e1 =
                   col + 1 < valid ? ex2(fmaf(__uint_as_float(sreg[qq][2 * c + 1]), p.scale_log2, nm)) : 0.f;
               ps[c & 7] += e0 + e1;
-              w[c] = pack_bf16_pos(e0, e1);
+              w[c] = pack_bf16(e0, e1);
             }
           }
           tmem_st16(sS + qq * 16, w);
         }
+      }
+      if constexpr (!C::kFused) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) ps[k] += ps2[k].x + ps2[k].y;
       }
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       // O_i rescale (PV_i(t-1) is complete, PV_i(t) not yet issued), done
