@@ -494,15 +494,8 @@ __global__ void __launch_bounds__(320, 1)
             for (int c = 0; c < 16; ++c) {
               const float2 a = __ffma2_rn(
                   make_float2(__uint_as_float(sreg[qq][2 * c]), __uint_as_float(sreg[qq][2 * c + 1])), sc2, nm2);
-              float e0, e1;
-              if (c % 3 == 2) {  // 5 of 16 pairs on the FMA pipe, the rest on MUFU
-                const float2 e = ex2_poly2(a.x, a.y);
-                e0 = e.x;
-                e1 = e.y;
-              } else {
-                e0 = ex2(a.x);
-                e1 = ex2(a.y);
-              }
+              const float e0 = ex2(a.x);
+              const float e1 = ex2(a.y);
               ps2[c & 3] = __fadd2_rn(ps2[c & 3], make_float2(e0, e1));
               w[c] = pack_bf16(e0, e1);
             }

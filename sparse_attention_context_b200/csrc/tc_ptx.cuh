@@ -221,40 +221,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA/ALU pipes, for x <= 126: x = n + f with n = rint(x) (by
-// adding 1.5 * 2^23, which leaves n in the low mantissa bits) and f in
-// [-0.5, 0.5]; 2^f from a cubic minimax polynomial fitted for this code by
-// Remez exchange (relative error 7.5e-5 in exact arithmetic, 1.5e-4 as
-// evaluated in fp32), then n is added to the exponent field.  Inputs below
-// -126 are clamped (result ~1e-38 instead of 0).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.05517166853f, f, 0.24261112511f), f, 0.69326096773f), f, 0.99992805719f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// ex2_poly on two values with packed fp32x2 arithmetic (same polynomial).
-__device__ __forceinline__ float2 ex2_poly2(float x0, float x1) {
-  const float2 x = make_float2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const float2 M = make_float2(12582912.f, 12582912.f);
-  const float2 t = __fadd2_rn(x, M);
-  const float2 f = __fadd2_rn(x, __fadd2_rn(M, make_float2(-t.x, -t.y)));
-  float2 pl = __ffma2_rn(make_float2(0.05517166853f, 0.05517166853f), f,
-                         make_float2(0.24261112511f, 0.24261112511f));
-  pl = __ffma2_rn(pl, f, make_float2(0.69326096773f, 0.69326096773f));
-  pl = __ffma2_rn(pl, f, make_float2(0.99992805719f, 0.99992805719f));
-  return make_float2(__int_as_float(__float_as_int(pl.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(pl.y) + (__float_as_int(t.y) << 23)));
-}
-
-// bf16x2 of two non-negative finite floats on the ALU pipe (round half up:
-// add half an ulp of bf16, keep the high halves); a in the low half.
-__device__ __forceinline__ uint32_t pack_bf16_pos(float a, float b) {
-  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
-}
-
 // max of three floats in one instruction (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
