@@ -143,6 +143,29 @@ int isa_taylor_attn_fwd(const isa_shape* shape, const uint16_t* q, const int32_t
 int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
+/* All four stages like isa_forward, for callers that cannot allocate device
+ * memory: frameworks whose caching allocator owns every free byte of the
+ * GPU, serving loops that must not allocate after start-up, or plugins that
+ * are handed tensors but no way to obtain scratch.  (The ISA pages have no
+ * counterpart; this is a packaging of the same path.)
+ * The scratch is a fixed array of ISA_STATIC_SCRATCH_BYTES inside this
+ * library; every GPU that loads the library holds it until the process
+ * exits.  Shapes whose isa_workspace_size() exceeds it (e.g. 40 heads of
+ * 75600 + 75600 tokens) return ISA_ERR_WORKSPACE without launching
+ * anything; invalid shapes return what isa_forward returns.  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream
+ * capture.  Each call clears the scratch's control block and calls
+ * isa_forward on it; nothing is allocated or freed.  All calls share the
+ * one array, which keeps the last call's contents: calls that overlap on
+ * the GPU (different streams, or different host threads on one device)
+ * race and corrupt each other.  The device status word of these calls is
+ * not readable by the caller; use isa_forward with an own workspace when
+ * device-side timeouts must be observed. */
+#define ISA_STATIC_SCRATCH_BYTES (64u << 20)
+int isa_forward_static(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       uint16_t* out, void* stream);
+
 /* In-house dense flash attention (the latency baseline; equals ISA at
  * keep = rho = 1): out = softmax(scale q k^T) v over all N keys, per (b, h),
  * non-causal.  scale <= 0 selects 1/sqrt(d).  ws: a zeroed buffer of

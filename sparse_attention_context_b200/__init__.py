@@ -8,7 +8,7 @@ binds that ABI for torch tensors.
 """
 from ._lib import IsaError, IsaShape, LIB_PATH, lib  # noqa: F401
 from .api import (  # noqa: F401
-    dense_workspace, isa_attn_fwd, isa_dense_attn_fwd, isa_forward, isa_full_attn_fwd, isa_n_keep, isa_n_route,
+    dense_workspace, isa_attn_fwd, isa_dense_attn_fwd, isa_forward, isa_forward_static, isa_full_attn_fwd, isa_n_keep, isa_n_route,
     isa_preselect_ctx, isa_read_device_status, isa_route_queries, isa_route_taylor_fwd, isa_selftest_umma,
     isa_taylor_attn_fwd,
     isa_workspace_size,

@@ -46,6 +46,7 @@ SIGNATURES = {
     "isa_full_attn_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_taylor_attn_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_forward": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
+    "isa_forward_static": (_I, [_SH, _P, _P, _P, _P, _P]),
     "isa_dense_workspace_size": (_SZ, [_I]),
     "isa_dense_attn_fwd": (_I, [_I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_read_device_status": (_I, [_P, _P]),

@@ -170,6 +170,20 @@ def isa_forward(q, k, v, N_src: int, block: int, keep: float, rho: float, scale:
     return o
 
 
+def isa_forward_static(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, out=None,
+                       stream=None):
+    """All ISA stages with the library's fixed device scratch (no workspace,
+    nothing allocated by the library).  CUDA tensors only; returns out."""
+    if out is None:
+        out = torch.empty_like(q)
+    _check_qkv(q, k, v, out)
+    shape = make_shape(q, N_src, block, keep, rho, scale)
+    rc = lib().isa_forward_static(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  _stream(stream))
+    check("isa_forward_static", rc)
+    return out
+
+
 def dense_workspace(d: int = 128, device="cuda") -> torch.Tensor:
     n = lib().isa_dense_workspace_size(int(d))
     if n == 0:
