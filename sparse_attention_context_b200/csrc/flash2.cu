@@ -90,12 +90,6 @@ __device__ __forceinline__ bool w1(uint64_t* bar, uint32_t par, Attn2Bars* bars,
   if (r == 2) raise2(bars, p);
   return r == 0;
 }
-// Polling variant for the issuing thread (reacts quickly to the softmax hand-off).
-__device__ __forceinline__ bool wpoll(uint64_t* bar, uint32_t par, Attn2Bars* bars, const FlashParams& p) {
-  const int r = mbar_poll_bounded(bar, par, reinterpret_cast<volatile int*>(&bars->abort), kWaitLimitNs);
-  if (r == 2) raise2(bars, p);
-  return r == 0;
-}
 __device__ __forceinline__ bool wwarp(uint64_t* bar, uint32_t par, Attn2Bars* bars, const FlashParams& p) {
   const bool ok = w1(bar, par, bars, p);
   return __all_sync(0xffffffffu, ok);
@@ -281,7 +275,7 @@ __global__ void __launch_bounds__(320, 1)
           // warpgroup has the other tile's PV and S (two MMAs) to hide behind.
           // S_i(t+1) overwrites the P_i(t) columns that PV_i(t), issued just
           // before it, reads: UMMAs issued by one thread execute in order.
-          if (!(ok = wpoll(&bars->p_full[0], ph, bars, p))) break;
+          if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
           tc_fence_after();
           issue_PV(0, t);
           if (more) {
@@ -289,7 +283,7 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             issue_S(0, t + 1);
           }
-          if (!(ok = wpoll(&bars->p_full[1], ph, bars, p))) break;
+          if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
           tc_fence_after();
           issue_PV(1, t);
           umma_commit(&bars->kv_empty[st]);
@@ -297,10 +291,10 @@ __global__ void __launch_bounds__(320, 1)
         } else {
           // One stage: K(t+1) lands only after PV(t) of both tiles released
           // the stage, so both PVs go first.
-          if (!(ok = wpoll(&bars->p_full[0], ph, bars, p))) break;
+          if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
           tc_fence_after();
           issue_PV(0, t);
-          if (!(ok = wpoll(&bars->p_full[1], ph, bars, p))) break;
+          if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
           tc_fence_after();
           issue_PV(1, t);
           umma_commit(&bars->kv_empty[st]);
@@ -481,7 +475,7 @@ __global__ void __launch_bounds__(320, 1)
               const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
               ps[(2 * c) & 7] += e0;
               ps[(2 * c + 1) & 7] += e1;
-              w[c] = pack_bf16(e0, e1);
+              w[c] = pack_bf16_pos(e0, e1);
             }
             tmem_st16(sS + h * 32 + j * 16, w);
           }
@@ -503,7 +497,7 @@ __global__ void __launch_bounds__(320, 1)
               const float e0 = ex2(a.x);
               const float e1 = ex2(a.y);
               ps2[c & 3] = __fadd2_rn(ps2[c & 3], make_float2(e0, e1));
-              w[c] = pack_bf16(e0, e1);
+              w[c] = pack_bf16_pos(e0, e1);
             }
           } else {
 #pragma unroll
@@ -513,7 +507,7 @@ __global__ void __launch_bounds__(320, 1)
               const float e1 =
                   col + 1 < valid ? ex2(fmaf(__uint_as_float(sreg[qq][2 * c + 1]), p.scale_log2, nm)) : 0.f;
               ps[c & 7] += e0 + e1;
-              w[c] = pack_bf16(e0, e1);
+              w[c] = pack_bf16_pos(e0, e1);
             }
           }
           tmem_st16(sS + qq * 16, w);

@@ -57,16 +57,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded polling wait: test_wait with a short sleep between probes, so a
-// single waiting thread notices the phase within ~tens of cycles while
-// leaving issue slots to the other warps of its SM sub-partition.
-// Returns 0 on success, 1 when *abort became non-zero, 2 on timeout.
-__device__ __forceinline__ int mbar_poll_bounded(uint64_t* bar, uint32_t parity, const volatile int* abort,
+// Bounded busy wait (test_wait, never suspends): for a single thread that
+// must react at once.  Returns 0 on success, 1 on abort, 2 on timeout.
+__device__ __forceinline__ int mbar_spin_bounded(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                                  uint64_t limit_ns) {
   if (mbar_test_wait(bar, parity)) return 0;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    __nanosleep(20);
     if (mbar_test_wait(bar, parity)) return 0;
     if (abort != nullptr && *abort) return 1;
     if (global_timer_ns() - t0 > limit_ns) return 2;
@@ -229,6 +226,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// bf16x2 of two non-negative finite floats on the integer pipe (round half
+// up: add half a bf16 ulp, keep the high halves), keeping the conversion
+// off the MUFU/XU pipe that the exponentials saturate; a in the low half.
+__device__ __forceinline__ uint32_t pack_bf16_pos(float a, float b) {
+  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
