@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(320, 1)
               const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
               ps[(2 * c) & 7] += e0;
               ps[(2 * c + 1) & 7] += e1;
-              w[c] = pack_bf16_pos(e0, e1);
+              w[c] = pack_bf16(e0, e1);
             }
             tmem_st16(sS + h * 32 + j * 16, w);
           }
@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(320, 1)
               const float e0 = ex2(a.x);
               const float e1 = ex2(a.y);
               ps2[c & 3] = __fadd2_rn(ps2[c & 3], make_float2(e0, e1));
-              w[c] = pack_bf16_pos(e0, e1);
+              w[c] = pack_bf16(e0, e1);
             }
           } else {
 #pragma unroll
@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(320, 1)
               const float e1 =
                   col + 1 < valid ? ex2(fmaf(__uint_as_float(sreg[qq][2 * c + 1]), p.scale_log2, nm)) : 0.f;
               ps[c & 7] += e0 + e1;
-              w[c] = pack_bf16_pos(e0, e1);
+              w[c] = pack_bf16(e0, e1);
             }
           }
           tmem_st16(sS + qq * 16, w);

@@ -228,13 +228,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// bf16x2 of two non-negative finite floats on the integer pipe (round half
-// up: add half a bf16 ulp, keep the high halves), keeping the conversion
-// off the MUFU/XU pipe that the exponentials saturate; a in the low half.
-__device__ __forceinline__ uint32_t pack_bf16_pos(float a, float b) {
-  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
