@@ -58,6 +58,22 @@ def counts(cfg):
     return nSB, nCB, n_keep, n_route
 
 
+def full_stage_launches(cfg, n_keep, n_route, nsm):
+    """Kernel launches of the routed full-attention stage: one launch for the
+    whole waves of 256-row items; when a partial last wave remains, its items
+    run split along the key tiles over the SMs (a second launch) and a combine
+    kernel merges the pieces (a third).  Mirrors the launcher's rule."""
+    if n_route <= 0:
+        return 0
+    nSB = -(-cfg.N_src // cfg.block)
+    items = cfg.B * cfg.H * (-(-n_route // 256))
+    rem = items % nsm
+    if rem == 0:
+        return 1
+    pieces = min(nsm // rem, (nSB + n_keep) // 4)
+    return 3 if pieces >= 2 else 1
+
+
 def work_model(cfg, kept_tokens_mean):
     """Executed FLOPs and algorithmic bytes of one step (all heads)."""
     nSB, nCB, n_keep, n_route = counts(cfg)
@@ -360,7 +376,8 @@ def main():
                "sample": f"{len(heads)} of {cfg.B * cfg.H} heads ({secs:.1f} s of CPU work), "
                          f"scaled x{cfg.B * cfg.H / len(heads):g}"}
 
-    launches_per_step = 3 + 3 + (1 if n_route > 0 else 0)
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    launches_per_step = 3 + 3 + full_stage_launches(cfg, n_keep, n_route, nsm)
     if rank == 0:
         rec = {"metric": METRIC, "value": round(ms_max, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": False,
