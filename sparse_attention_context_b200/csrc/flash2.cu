@@ -33,6 +33,9 @@
 //
 // Ordering: the issuer runs the tensor pipe as PV0(t), S0(t+1), PV1(t),
 // S1(t+1), so each tile's softmax overlaps two MMAs of the other tile.
+// The softmax hands P_i(t) over in parts of 32 keys (one mbarrier each);
+// the issuer starts PV_i(t) on the first part while the later ones are
+// still being exponentiated, so the tensor pipe waits only for the last.
 // S_i(t+1) overwrites the columns PV_i(t) reads as P_i(t); it is issued
 // behind PV_i(t) by the same thread and UMMAs from one thread execute in
 // order.  The commit that signals S_i(t+1) fires only when every earlier
@@ -55,6 +58,10 @@ struct Attn2Cfg {
   static constexpr int Q_BYTES = TILE * D * 2;      // one tile
   static constexpr int KT_BYTES = BN * D * 2;       // one key (or value) tile
   static constexpr int NKT = kFused ? 3 : 2;        // tiles per stage: K[,Klo],V
+  // P hand-off in parts of 32 keys (one barrier each), so PV starts on the
+  // first keys while the softmax still exponentiates the rest; FUSED hands
+  // its P over whole.
+  static constexpr int NP = kFused ? 1 : BN / 32;
   static constexpr int STAGE_BYTES = NKT * KT_BYTES;
   static constexpr int BUDGET = 225 * 1024;
   static constexpr int ST_FIT = (BUDGET - 2 * Q_BYTES - 1024 - 256) / STAGE_BYTES;
@@ -74,7 +81,7 @@ struct Attn2Bars {
   uint64_t v_full[3];
   uint64_t kv_empty[3];
   uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t p_part[2][4];
   uint64_t o_done[2];
   uint64_t teardown;
   uint32_t tmem_base;
@@ -154,7 +161,7 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->q_full[i], C::kTmaQ ? 1 : 128);
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
+      for (int q = 0; q < 4; ++q) mbar_init(&bars->p_part[i][q], 128);
       mbar_init(&bars->o_done[i], 1);
     }
     for (int s = 0; s < 3; ++s) {
@@ -248,14 +255,24 @@ __global__ void __launch_bounds__(320, 1)
         }
         umma_commit(&bars->s_full[i]);
       };
-      auto issue_PV = [&](int i, int t) {
+      // PV_i(t), part by part as the softmax hands P over (false: a wait gave up)
+      auto issue_PV = [&](int i, int t) -> bool {
         const int st = t % ST;
         const uint32_t vb = aKV + st * C::STAGE_BYTES + (C::NKT - 1) * C::KT_BYTES;
+        constexpr int KS = BN / 16 / C::NP;  // k-steps per part
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_tmem_a(tmem + 2 * BN + i * D, tmem + i * BN + kk * 8, desc_mn_sw128(vb + kk * 16 * 128, BN * 128),
-                           IDO, (t > 0 || kk > 0) ? 1u : 0u);
+        for (int qp = 0; qp < C::NP; ++qp) {
+          if (!w1(&bars->p_part[i][qp], t & 1, bars, p)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k2 = 0; k2 < KS; ++k2) {
+            const int kk = qp * KS + k2;
+            umma_bf16_tmem_a(tmem + 2 * BN + i * D, tmem + i * BN + kk * 8,
+                             desc_mn_sw128(vb + kk * 16 * 128, BN * 128), IDO, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
         umma_commit(&bars->o_done[i]);
+        return true;
       };
       if (ok && nT > 0) {
         ok = w1(&bars->k_full[0], 0, bars, p);
@@ -267,7 +284,6 @@ __global__ void __launch_bounds__(320, 1)
       }
       for (int t = 0; ok && t < nT; ++t) {
         const int st = t % ST;
-        const uint32_t ph = t & 1;
         const bool more = t + 1 < nT;
         if (!(ok = w1(&bars->v_full[st], (t / ST) & 1, bars, p))) break;
         if constexpr (ST >= 2) {
@@ -275,28 +291,20 @@ __global__ void __launch_bounds__(320, 1)
           // warpgroup has the other tile's PV and S (two MMAs) to hide behind.
           // S_i(t+1) overwrites the P_i(t) columns that PV_i(t), issued just
           // before it, reads: UMMAs issued by one thread execute in order.
-          if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
-          tc_fence_after();
-          issue_PV(0, t);
+          if (!(ok = issue_PV(0, t))) break;
           if (more) {
             if (!(ok = w1(&bars->k_full[(t + 1) % ST], ((t + 1) / ST) & 1, bars, p))) break;
             tc_fence_after();
             issue_S(0, t + 1);
           }
-          if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
-          tc_fence_after();
-          issue_PV(1, t);
+          if (!(ok = issue_PV(1, t))) break;
           umma_commit(&bars->kv_empty[st]);
           if (more) issue_S(1, t + 1);
         } else {
           // One stage: K(t+1) lands only after PV(t) of both tiles released
           // the stage, so both PVs go first.
-          if (!(ok = w1(&bars->p_full[0], ph, bars, p))) break;
-          tc_fence_after();
-          issue_PV(0, t);
-          if (!(ok = w1(&bars->p_full[1], ph, bars, p))) break;
-          tc_fence_after();
-          issue_PV(1, t);
+          if (!(ok = issue_PV(0, t))) break;
+          if (!(ok = issue_PV(1, t))) break;
           umma_commit(&bars->kv_empty[st]);
           if (more) {
             if (!(ok = w1(&bars->k_full[0], ((t + 1) / ST) & 1, bars, p))) break;
@@ -449,9 +457,13 @@ __global__ void __launch_bounds__(320, 1)
       }
       mx = fmaxf(mx, mt);
       const float m_new = fmaxf(m, mt);
-      // Rescale only when the running maximum grew by more than 2^8: the
-      // stale reference keeps every p <= 256, exact after the final 1/l.
-      const bool need = m_new > m + 8.0f;
+      // Rescale only when the running maximum grew by more than 2^32: with
+      // the stale reference every p stays <= 2^32 (bf16 and fp32 hold that
+      // with the same relative precision; l <= n_keys * 2^32 is far from
+      // fp32 overflow) and the result is exact after the final 1/l.  A small
+      // threshold would make some warp rescale O on most key tiles when the
+      // logits span tens of units (sharp routed queries).
+      const bool need = m_new > m + 32.0f;
       // factor for the accumulated O and l when the reference moves
       const float alpha = need ? ex2(m - m_new) : 1.f;
       if (need) {
@@ -511,6 +523,25 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
           tmem_st16(sS + qq * 16, w);
+          if (qq == 0 && t > 0 && __any_sync(0xffffffffu, need)) {
+            // O_i rescale (PV_i(t-1) is complete, no part of PV_i(t) issued
+            // yet), once the first quarter's scores have left the registers;
+            // 16 columns at a time beside the 96 scores still held
+#pragma unroll 1
+            for (int j = 0; j < D / 16; ++j) {
+              uint32_t u[16];
+              tmem_ld16(sO + j * 16, u);
+              tmem_wait_ld();
+              regs_after(u);
+#pragma unroll
+              for (int c = 0; c < 16; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+              tmem_st16(sO + j * 16, u);
+            }
+          }
+          // hand P columns [16q, 16q+16) to the issuer
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bars->p_part[i][qq]);
         }
       }
       if constexpr (!C::kFused) {
@@ -518,23 +549,25 @@ __global__ void __launch_bounds__(320, 1)
         for (int k = 0; k < 4; ++k) ps[k] += ps2[k].x + ps2[k].y;
       }
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      // O_i rescale (PV_i(t-1) is complete, PV_i(t) not yet issued), done
-      // after the scores left the registers
-      if (t > 0 && __any_sync(0xffffffffu, need)) {
+      if constexpr (C::kFused) {
+        // O_i rescale (PV_i(t-1) is complete, PV_i(t) not yet issued), done
+        // after the logits left the registers; then P goes over whole
+        if (t > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
-          uint32_t u[32];
-          tmem_ld32(sO + j * 32, u);
-          tmem_wait_ld();
-          regs_after(u);
+          for (int j = 0; j < D / 32; ++j) {
+            uint32_t u[32];
+            tmem_ld32(sO + j * 32, u);
+            tmem_wait_ld();
+            regs_after(u);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
-          tmem_st32(sO + j * 32, u);
+            for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+            tmem_st32(sO + j * 32, u);
+          }
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_part[i][0]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[i]);
     }
 
     const bool valid_row = g < p.n_rows;
