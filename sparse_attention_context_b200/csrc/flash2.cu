@@ -79,7 +79,8 @@ struct Attn2Bars {
   uint64_t q_full[2];
   uint64_t k_full[3];
   uint64_t v_full[3];
-  uint64_t kv_empty[3];
+  uint64_t k_empty[3];  // K slot free: S_1 of its tile done
+  uint64_t v_empty[3];  // V slot free: PV_1 of its tile done
   uint64_t s_full[2];
   uint64_t p_part[2][4];
   uint64_t o_done[2];
@@ -167,7 +168,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < 3; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->teardown, 1);
     bars->abort = 0;
@@ -203,7 +205,9 @@ __global__ void __launch_bounds__(320, 1)
       int issued = 0;
       for (int t = 0; t < nT; ++t) {
         const int st = t % ST;
-        if (t >= ST && !w1(&bars->kv_empty[st], ((t / ST) - 1) & 1, bars, p)) break;
+        // K and V slots are released separately: K(t) is last read by
+        // S_1(t), V(t) by PV_1(t) two MMAs later, so K(t + ST) loads early
+        if (t >= ST && !w1(&bars->k_empty[st], ((t / ST) - 1) & 1, bars, p)) break;
         const int r = kv_row<BN, MODE>(p, bh, kv0 + t);
         uint8_t* base = smem + C::OFF_KV + st * C::STAGE_BYTES;
         mbar_arrive_expect_tx(&bars->k_full[st], (C::kFused ? 2 : 1) * C::KT_BYTES);
@@ -215,6 +219,7 @@ __global__ void __launch_bounds__(320, 1)
             tma_load_2d(base + C::KT_BYTES + c * (BN * 128), &tmK2, &bars->k_full[st], c * 64, r);
         }
         uint8_t* vb = base + (C::NKT - 1) * C::KT_BYTES;
+        if (t >= ST && !w1(&bars->v_empty[st], ((t / ST) - 1) & 1, bars, p)) break;
         mbar_arrive_expect_tx(&bars->v_full[st], C::KT_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) tma_load_2d(vb + c * (BN * 128), &tmV, &bars->v_full[st], c * 64, r);
@@ -280,6 +285,7 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
           issue_S(0, 0);
           issue_S(1, 0);
+          umma_commit(&bars->k_empty[0]);
         }
       }
       for (int t = 0; ok && t < nT; ++t) {
@@ -298,19 +304,23 @@ __global__ void __launch_bounds__(320, 1)
             issue_S(0, t + 1);
           }
           if (!(ok = issue_PV(1, t))) break;
-          umma_commit(&bars->kv_empty[st]);
-          if (more) issue_S(1, t + 1);
+          umma_commit(&bars->v_empty[st]);
+          if (more) {
+            issue_S(1, t + 1);
+            umma_commit(&bars->k_empty[(t + 1) % ST]);
+          }
         } else {
-          // One stage: K(t+1) lands only after PV(t) of both tiles released
-          // the stage, so both PVs go first.
+          // One stage: V(t+1) lands only after PV(t) of both tiles released
+          // its slot, so both PVs go first (K(t+1) loads once S_1(t) is done).
           if (!(ok = issue_PV(0, t))) break;
           if (!(ok = issue_PV(1, t))) break;
-          umma_commit(&bars->kv_empty[st]);
+          umma_commit(&bars->v_empty[st]);
           if (more) {
             if (!(ok = w1(&bars->k_full[0], ((t + 1) / ST) & 1, bars, p))) break;
             tc_fence_after();
             issue_S(0, t + 1);
             issue_S(1, t + 1);
+            umma_commit(&bars->k_empty[0]);
           }
         }
       }
@@ -506,10 +516,15 @@ __global__ void __launch_bounds__(320, 1)
             for (int c = 0; c < 16; ++c) {
               const float2 a = __ffma2_rn(
                   make_float2(__uint_as_float(sreg[qq][2 * c]), __uint_as_float(sreg[qq][2 * c + 1])), sc2, nm2);
-              const float e0 = ex2(a.x);
-              const float e1 = ex2(a.y);
-              ps2[c & 3] = __fadd2_rn(ps2[c & 3], make_float2(e0, e1));
-              w[c] = pack_bf16(e0, e1);
+              float2 e;
+              if (c % 3 == 2) {  // 5 of 16 pairs on the FMA pipe, the rest on MUFU
+                e = ex2_poly2(a);
+              } else {
+                e.x = ex2(a.x);
+                e.y = ex2(a.y);
+              }
+              ps2[c & 3] = __fadd2_rn(ps2[c & 3], e);
+              w[c] = pack_bf16(e.x, e.y);
             }
           } else {
 #pragma unroll
@@ -521,6 +536,13 @@ __global__ void __launch_bounds__(320, 1)
               ps[c & 7] += e0 + e1;
               w[c] = pack_bf16(e0, e1);
             }
+          }
+          // hand the previous quarter's P to the issuer: its store has had
+          // this quarter's exponentials to complete
+          if (qq > 0) {
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_part[i][qq - 1]);
           }
           tmem_st16(sS + qq * 16, w);
           if (qq == 0 && t > 0 && __any_sync(0xffffffffu, need)) {
@@ -538,11 +560,10 @@ __global__ void __launch_bounds__(320, 1)
               tmem_st16(sO + j * 16, u);
             }
           }
-          // hand P columns [16q, 16q+16) to the issuer
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&bars->p_part[i][qq]);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_part[i][BN / 32 - 1]);
       }
       if constexpr (!C::kFused) {
 #pragma unroll

@@ -141,6 +141,32 @@ __device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tme
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same two UMMA forms with the shared-memory descriptors given as their
+// 32-bit halves: `*_lo` carries the start address >> 4 (bits 0-13) and the
+// leading byte offset >> 4 (bits 16-29), `hi` the stride byte offset >> 4,
+// the version bit and the swizzle mode (see smem_desc).  An issuing loop can
+// then step through K by adding (bytes >> 4) to a precomputed low half.
+__device__ __forceinline__ void umma_bf16_lohi(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 da, {%1, %3};\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_tmem_a_lohi(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                                      uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 db, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(hi)
+      : "memory");
+}
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -203,6 +229,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   d |= static_cast<uint64_t>(2) << 61;
   return d;
 }
+// Halves of smem_desc (for the *_lohi UMMA forms).
+__host__ __device__ constexpr uint32_t desc_hi_sw128(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
 // K-major operand in 128B-swizzled atoms (rows of 128 bytes, 8-row groups
 // 1024 bytes apart).  The leading offset is unused for this layout.
 __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) { return smem_desc(saddr, 16, 1024); }
@@ -227,6 +260,28 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for two values on the FMA pipe, packed fp32x2 (relieves the MUFU
+// pipe, which the exponentials of a softmax otherwise saturate).  Method:
+// Cody-Waite range reduction x = n + f, n = rint(x) by the 1.5*2^23
+// round-to-integer addition, f in [-0.5, 0.5]; 2^f by a cubic with
+// coefficients from a Remez exchange for minimal relative error on that
+// interval (max relative error 7.5e-5, 1.5e-4 in fp32 arithmetic, below
+// the 2^-9 of the bf16 rounding that follows); 2^n applied by
+// adding n to the exponent field.  x is clamped at -126 so that the result
+// stays a normal float (2^-126 is far below anything a softmax keeps).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+  const float2 M = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, M);                                     // n in t's low mantissa bits
+  const float2 f = __fadd2_rn(x, __fadd2_rn(M, make_float2(-t.x, -t.y)));  // x - n
+  float2 q = __ffma2_rn(make_float2(0.05517166853f, 0.05517166853f), f,
+                        make_float2(0.24261112511f, 0.24261112511f));
+  q = __ffma2_rn(q, f, make_float2(0.69326096773f, 0.69326096773f));
+  q = __ffma2_rn(q, f, make_float2(0.99992805719f, 0.99992805719f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 // max of three floats in one instruction (sm_100).
