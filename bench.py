@@ -58,6 +58,35 @@ def counts(cfg):
     return nSB, nCB, n_keep, n_route
 
 
+# DRAM bytes (read + write) of one routed full-attention stage at the 480p
+# workload -- whole-wave launch, key-split launch and combine -- summed from
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass).
+# They hold only for the kernel sources they were taken on: on any other
+# source, or another workload, the report's traffic is null.
+FULL_TRAFFIC = {
+    "config": "480p",
+    "bytes": 387_516_672 + 37_400_064 + 15_112_960 + 11_520 + 18_467_328,
+    "sources": {
+        "sparse_attention_context_b200/csrc/flash2.cu": "6e65216d95f4e63af94970034b00c2b978e01593ead2f49c1bc3fb718ca7f816",
+        "sparse_attention_context_b200/csrc/tc_ptx.cuh": "014a3c466b7859b30d53c5e121984b9e032b9ddec01309fde00c3151e40b0a26",
+    },
+}
+
+
+def full_traffic(args):
+    """The captured stage traffic if it applies to this run, else None."""
+    import hashlib
+
+    if args.config != FULL_TRAFFIC["config"] or args.heads or args.rho is not None or args.keep is not None:
+        return None
+    root = os.path.dirname(os.path.abspath(__file__))
+    for rel, digest in FULL_TRAFFIC["sources"].items():
+        with open(os.path.join(root, rel), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None
+    return FULL_TRAFFIC["bytes"]
+
+
 def full_stage_launches(cfg, n_keep, n_route, nsm):
     """Kernel launches of the routed full-attention stage: one launch for the
     whole waves of 256-row items; when a partial last wave remains, its items
@@ -359,7 +388,8 @@ def main():
             "achieved": round(ach, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
             "frac": round(ach / pk["bf16_tflops"], 4), "peak_kind": f"{pk_kind} burst bf16",
             "frac_of_sustained": round(ach / pk["bf16_tflops_sustained"], 4),
-            "traffic": None, "kernel_ms": round(full_ms, 4)}
+            "traffic": full_traffic(args), "algorithmic_bytes": int(wm["full_bytes"]),
+            "kernel_ms": round(full_ms, 4)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
