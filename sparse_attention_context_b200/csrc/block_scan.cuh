@@ -30,4 +30,32 @@ __device__ __forceinline__ int block_rank_1024(bool flag, int* ws, int& total) {
   return off + in_warp;
 }
 
+// Exclusive prefix sum of `v` over the CTA in thread order; `total`
+// receives the CTA-wide sum.  Same calling rules as block_rank_1024.
+__device__ __forceinline__ int block_exclusive_sum_1024(int v, int* ws, int& total) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) ws[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int t = ws[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += n;
+    }
+    ws[lane] = t;  // inclusive over warps
+  }
+  __syncthreads();
+  const int off = w ? ws[w - 1] : 0;
+  total = ws[31];
+  __syncthreads();  // ws may be reused right after
+  return off + incl - v;
+}
+
 }  // namespace isa
