@@ -12,7 +12,7 @@ constexpr int kStatusOffset = 0;   // int32 in the workspace control block
 constexpr int kInjectOffset = 4;   // int32 fault-injection word (tests)
 constexpr int kCtlBytes = 256;
 constexpr int kTopkCap = 4096;     // max context blocks the top-k sort holds
-constexpr int kSalRows = 16;       // query blocks per saliency CTA
+constexpr int kSalRows = 32;       // query blocks per saliency CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
 enum FlashMode { MODE_DENSE = 0, MODE_FULL = 1, MODE_TAYLOR = 2, MODE_SHARP = 3, MODE_FUSED = 4 };

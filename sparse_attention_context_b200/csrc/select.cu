@@ -9,10 +9,11 @@
 // n_keep most salient context blocks are kept (higher saliency first, lower
 // block number on ties), every source block is always kept.
 //
-// saliency_kernel: grid (ceil(nB/16), B*H); a CTA owns 16 query blocks,
-//   computes their logits against every key block in fp32 (two passes: row
-//   max and sum, then the column contributions; logits recomputed bit-
-//   identically), and writes per-chunk partial column sums.
+// saliency_kernel: grid (ceil(nB/32), B*H); a CTA owns 32 query blocks and
+//   walks the key blocks in tiles of 64 staged in shared memory (each K-bar
+//   row is read from L2 once per pass per CTA), computing the logits in fp32
+//   (two passes: row max and sum, then the column contributions; logits
+//   recomputed bit-identically), and writes per-chunk partial column sums.
 // select_ctx_kernel: one 1024-thread CTA per (b, h); sums the partials in a
 //   fixed order, bitonic-sorts (saliency, block) keys in shared memory, and
 //   writes the kept block numbers in ascending order.
@@ -32,111 +33,141 @@ __device__ __forceinline__ int block_count(int b, int nSB, int N_src, int N_ctx,
   return b < nSB ? min(blk, N_src - b * blk) : min(blk, N_ctx - (b - nSB) * blk);
 }
 
+// Shared-memory tile sizes of saliency_kernel.
+constexpr int kSalColTile = 64;  // key blocks staged per tile
+template <int D>
+constexpr int sal_smem_bytes() {
+  return (kSalRows * D + kSalColTile * (D + 4) + 16 * kSalColTile) * 4;
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) saliency_kernel(const float* __restrict__ Qbar, const float* __restrict__ Kbar,
                                                        float* __restrict__ partial, int N_src, int N_ctx, int blk,
                                                        int nSB, int nB, float scale) {
-  constexpr int RB = kSalRows;
-  __shared__ __align__(16) float sQ[RB][D];
-  __shared__ float red[RB][8];
-  __shared__ float rowM[RB], rowS[RB];
-  const int chunk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  constexpr int RB = kSalRows;     // query blocks of this CTA
+  constexpr int CT = kSalColTile;  // key blocks per staged tile
+  constexpr int KP = D + 4;        // padded row of the staged tile (conflict-free float4 columns)
+  extern __shared__ __align__(16) float sal_sm[];
+  float* sQ = sal_sm;               // [RB][D]
+  float* sK = sQ + RB * D;          // [CT][KP]
+  float* sRed = sK + CT * KP;       // [16][CT] column partial sums of the 16 row pairs
+  const int chunk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;  // rows 2ty, 2ty+1; tile columns tx + 16m
   const int nCB = nB - nSB;
   const int r0 = chunk * RB;
   const int nr = min(RB, nB - r0);
-  for (int e = tid; e < RB * D; e += 256) {
-    const int rr = e / D, col = e % D;
-    sQ[rr][col] = rr < nr ? Qbar[(static_cast<size_t>(bh) * nB + r0 + rr) * D + col] : 0.f;
-  }
-  __syncthreads();
   const float* Kh = Kbar + static_cast<size_t>(bh) * nB * D;
-
-  auto logits = [&](int c, float (&lg)[RB]) {
-    float acc[RB];
+  for (int e = tid; e < RB * D / 4; e += 256) {
+    const int rr = e / (D / 4), q4 = e % (D / 4);
+    const float4 v = rr < nr ? __ldg(reinterpret_cast<const float4*>(Qbar + (static_cast<size_t>(bh) * nB + r0 + rr) * D) + q4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(sQ + rr * D + 4 * q4) = v;
+  }
+  // K rows [c0, c0 + CT) into sK (zero past nB); the caller syncs around it
+  auto stage = [&](int c0) {
+    for (int e = tid; e < CT * D / 4; e += 256) {
+      const int rr = e / (D / 4), q4 = e % (D / 4);
+      const int c = c0 + rr;
+      const float4 v = c < nB ? __ldg(reinterpret_cast<const float4*>(Kh + static_cast<size_t>(c) * D) + q4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(sK + rr * KP + 4 * q4) = v;
+    }
+  };
+  // logits of rows 2ty, 2ty+1 against tile columns tx + 16m (-inf past nB);
+  // each dot product accumulates over d in order, as a plain loop would
+  auto tile_logits = [&](int c0, float (&lg)[2][4]) {
+    float acc[2][4];
 #pragma unroll
-    for (int rr = 0; rr < RB; ++rr) acc[rr] = 0.f;
-    const float4* kc = reinterpret_cast<const float4*>(Kh + static_cast<size_t>(c) * D);
-#pragma unroll 4
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[i][m] = 0.f;
+#pragma unroll 8
     for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 kv = __ldg(kc + d4);
+      const float4 qa = *reinterpret_cast<const float4*>(sQ + (2 * ty) * D + 4 * d4);
+      const float4 qb = *reinterpret_cast<const float4*>(sQ + (2 * ty + 1) * D + 4 * d4);
 #pragma unroll
-      for (int rr = 0; rr < RB; ++rr) {
-        const float4 qv = *reinterpret_cast<const float4*>(&sQ[rr][4 * d4]);
-        acc[rr] = fmaf(qv.x, kv.x, acc[rr]);
-        acc[rr] = fmaf(qv.y, kv.y, acc[rr]);
-        acc[rr] = fmaf(qv.z, kv.z, acc[rr]);
-        acc[rr] = fmaf(qv.w, kv.w, acc[rr]);
+      for (int m = 0; m < 4; ++m) {
+        const float4 kv = *reinterpret_cast<const float4*>(sK + (tx + 16 * m) * KP + 4 * d4);
+        acc[0][m] = fmaf(qa.x, kv.x, acc[0][m]);
+        acc[0][m] = fmaf(qa.y, kv.y, acc[0][m]);
+        acc[0][m] = fmaf(qa.z, kv.z, acc[0][m]);
+        acc[0][m] = fmaf(qa.w, kv.w, acc[0][m]);
+        acc[1][m] = fmaf(qb.x, kv.x, acc[1][m]);
+        acc[1][m] = fmaf(qb.y, kv.y, acc[1][m]);
+        acc[1][m] = fmaf(qb.z, kv.z, acc[1][m]);
+        acc[1][m] = fmaf(qb.w, kv.w, acc[1][m]);
       }
     }
-    const float lc = logf(static_cast<float>(block_count(c, nSB, N_src, N_ctx, blk)));
 #pragma unroll
-    for (int rr = 0; rr < RB; ++rr) lg[rr] = fmaf(scale, acc[rr], lc);
+    for (int m = 0; m < 4; ++m) {
+      const int c = c0 + tx + 16 * m;
+      const float lc = c < nB ? logf(static_cast<float>(block_count(c, nSB, N_src, N_ctx, blk))) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) lg[i][m] = c < nB ? fmaf(scale, acc[i][m], lc) : -INFINITY;
+    }
   };
 
-  // Pass 1: per-row max and sum of exp over all key blocks.
-  float mloc[RB], sloc[RB];
+  // Pass 1: max and sum of exp of each row over all key blocks (online per
+  // thread over its columns, then merged across the 16 threads of a row pair)
+  float rm[2] = {-INFINITY, -INFINITY}, rs[2] = {0.f, 0.f};
+  for (int c0 = 0; c0 < nB; c0 += CT) {
+    __syncthreads();
+    stage(c0);
+    __syncthreads();
+    float lg[2][4];
+    tile_logits(c0, lg);
 #pragma unroll
-  for (int rr = 0; rr < RB; ++rr) {
-    mloc[rr] = -INFINITY;
-    sloc[rr] = 0.f;
-  }
-  for (int c = tid; c < nB; c += 256) {
-    float lg[RB];
-    logits(c, lg);
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int rr = 0; rr < RB; ++rr) {
-      const float mn = fmaxf(mloc[rr], lg[rr]);
-      sloc[rr] = sloc[rr] * expf(mloc[rr] - mn) + expf(lg[rr] - mn);
-      mloc[rr] = mn;
-    }
+      for (int m = 0; m < 4; ++m) {
+        const float mn = fmaxf(rm[i], lg[i][m]);
+        if (mn != -INFINITY) {
+          rs[i] = rs[i] * expf(rm[i] - mn) + expf(lg[i][m] - mn);
+          rm[i] = mn;
+        }
+      }
   }
 #pragma unroll
-  for (int rr = 0; rr < RB; ++rr) {
-    float mm = mloc[rr];
+  for (int i = 0; i < 2; ++i) {
+    float mm = rm[i];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
-    float ss = (mloc[rr] == -INFINITY) ? 0.f : sloc[rr] * expf(mloc[rr] - mm);
+    for (int o = 8; o; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+    float ss = rm[i] == -INFINITY ? 0.f : rs[i] * expf(rm[i] - mm);
 #pragma unroll
-    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) {
-      red[rr][w] = mm;
-      rowS[rr] = 0.f;
-    }
-    mloc[rr] = mm;
-    sloc[rr] = ss;
+    for (int o = 8; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    rm[i] = mm;
+    rs[i] = ss;
   }
-  __syncthreads();
-  if (tid < RB) {
-    float mm = -INFINITY;
-    for (int i = 0; i < 8; ++i) mm = fmaxf(mm, red[tid][i]);
-    rowM[tid] = mm;
-  }
-  __syncthreads();
+  // weight of each row: cnt_r / S_r (zero for rows past the last block)
+  float wr[2];
 #pragma unroll
-  for (int rr = 0; rr < RB; ++rr) {
-    if (lane == 0) red[rr][w] = sloc[rr] * expf(mloc[rr] - rowM[rr]);
+  for (int i = 0; i < 2; ++i) {
+    const int r = 2 * ty + i;
+    wr[i] = r < nr ? static_cast<float>(block_count(r0 + r, nSB, N_src, N_ctx, blk)) / rs[i] : 0.f;
   }
-  __syncthreads();
-  if (tid < RB) {
-    float ss = 0.f;
-    for (int i = 0; i < 8; ++i) ss += red[tid][i];
-    rowS[tid] = ss;
-  }
-  __syncthreads();
 
-  // Pass 2: column contributions sum_r cnt_r * P_rc for context blocks.
-  float wr[RB];
-#pragma unroll
-  for (int rr = 0; rr < RB; ++rr)
-    wr[rr] = rr < nr ? static_cast<float>(block_count(r0 + rr, nSB, N_src, N_ctx, blk)) / rowS[rr] : 0.f;
+  // Pass 2: column contributions sum_r cnt_r * P_rc for the context blocks
   float* out = partial + (static_cast<size_t>(bh) * gridDim.x + chunk) * nCB;
-  for (int c = nSB + tid; c < nB; c += 256) {
-    float lg[RB];
-    logits(c, lg);
-    float col = 0.f;
+  for (int c0 = nSB; c0 < nB; c0 += CT) {
+    __syncthreads();
+    stage(c0);
+    __syncthreads();
+    float lg[2][4];
+    tile_logits(c0, lg);
 #pragma unroll
-    for (int rr = 0; rr < RB; ++rr) col = fmaf(wr[rr], expf(lg[rr] - rowM[rr]), col);
-    out[c - nSB] = col;
+    for (int m = 0; m < 4; ++m) {
+      float col = 0.f;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) col = fmaf(wr[i], expf(lg[i][m] - rm[i]), col);
+      sRed[ty * CT + tx + 16 * m] = col;
+    }
+    __syncthreads();
+    if (tid < CT && c0 + tid < nB) {
+      float col = 0.f;
+#pragma unroll
+      for (int y = 0; y < 16; ++y) col += sRed[y * CT + tid];
+      out[c0 + tid - nSB] = col;
+    }
   }
 }
 
@@ -242,10 +273,18 @@ cudaError_t launch_saliency(const float* Qbar, const float* Kbar, float* partial
   const int nSB = (N_src + blk - 1) / blk, nCB = (N_ctx + blk - 1) / blk, nB = nSB + nCB;
   if (nCB == 0) return cudaSuccess;
   const dim3 grid((nB + kSalRows - 1) / kSalRows, BH);
-  if (D == 128)
-    saliency_kernel<128><<<grid, 256, 0, st>>>(Qbar, Kbar, partial, N_src, N_ctx, blk, nSB, nB, scale);
-  else
-    saliency_kernel<64><<<grid, 256, 0, st>>>(Qbar, Kbar, partial, N_src, N_ctx, blk, nSB, nB, scale);
+  cudaError_t e;
+  if (D == 128) {
+    constexpr int smem = sal_smem_bytes<128>();
+    if ((e = cudaFuncSetAttribute(saliency_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    saliency_kernel<128><<<grid, 256, smem, st>>>(Qbar, Kbar, partial, N_src, N_ctx, blk, nSB, nB, scale);
+  } else {
+    constexpr int smem = sal_smem_bytes<64>();
+    if ((e = cudaFuncSetAttribute(saliency_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    saliency_kernel<64><<<grid, 256, smem, st>>>(Qbar, Kbar, partial, N_src, N_ctx, blk, nSB, nB, scale);
+  }
   return cudaGetLastError();
 }
 
