@@ -203,8 +203,33 @@ def cpu_oracle_ms_per_step(cfg, heads, seed=0):
     return 1e3 * t_total / len(heads) * cfg.B * cfg.H, t_total
 
 
+def dist_env():
+    """(world size, rank, local rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x, device):
+    """Max of a per-rank float over all ranks of the default process group
+    (the value itself on one rank).  Timing only: never on the data path."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(rank):
+    """Each rank's replica of the workload draws its own inputs (weak scaling:
+    every (b, h) of every replica is an independent unit)."""
+    return rank
+
+
 def run_reference(args, cfg):
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = dist_env()
     if rank != 0:
         return
     cores = len(os.sched_getaffinity(0))
@@ -264,9 +289,7 @@ def main():
 
     from sparse_attention_context_b200 import api
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     if world > 1:
         import datetime
 
@@ -280,7 +303,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    bits = make_inputs(cfg, seed=rank)
+    bits = make_inputs(cfg, seed=replica_seed(rank))
     q, k, v = (to_torch_bf16(b).to(dev) for b in bits)
     shape = api.make_shape(q, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     ws = api.new_workspace(shape, dev)
@@ -331,11 +354,7 @@ def main():
     ms = t0.elapsed_time(t1) / args.steps
     stage_ms = np.array([[stage_ev[i][j].elapsed_time(stage_ev[i][j + 1]) for j in range(3)]
                          for i in range(args.steps)]).mean(axis=0)
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
     assert api.isa_read_device_status(ws) == 0
 
     # in-house dense kernel on the same inputs (the baseline the metric names)
@@ -373,11 +392,7 @@ def main():
             api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws, out=hout)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / ne
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / ne, dev)
         e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": 3 * q.numel() * 2,
                "d2h_bytes_per_step": q.numel() * 2}
 
