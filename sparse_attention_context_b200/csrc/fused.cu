@@ -1,0 +1,454 @@
+// fused.cu -- persistent tcgen05 kernel for ISA sharpness + 0-th order
+// Taylor attention over every query (stages 2 and 4 in one pass).
+//
+// Method ("Lightning Unified Video Editing via In-Context Sparse Attention",
+// abstract): a query's sharpness is the largest probability of its block
+// distribution over the kept blocks, and the queries that are not routed to
+// full attention get the 0-th order Taylor output, whose keys and values
+// are the block means.  Both come from the same logits
+//   l_ib = s * q_i . Kbar_b + log cnt_b   over the kept blocks b:
+//   sharp_i = max_b softmax_b(l_i)  and  o_i = softmax_b(l_i) . Vbar.
+// The logits use Kbar split as bf16 hi + lo (two UMMAs, fp32-grade) so the
+// routing decision matches a float64 evaluation; the log2 cnt key biases
+// (-inf on padding) are read per key tile; Vbar is the bf16 V operand.
+//
+// A work item is 256 query rows of one (b, h) (two 128-row tiles) against
+// the head's nK_pad gathered kept blocks (a few 128-key tiles).  With so few
+// key tiles per item, a CTA per item spends most of its life loading Q from
+// HBM and storing O, one CTA per SM.  Here one CTA per SM loops over items
+// (stride = grid size): Q of the next item is loaded into a second buffer
+// while the current item computes, and the epilogue (O from TMEM to HBM) of
+// one item overlaps the QK^T products of the next.
+//
+// Warps (320 threads): 0-3 softmax of tile 0, 4-7 tile 1 (thread <-> query
+// row <-> TMEM lane), 8 TMA producer, 9 TMEM allocator + the single UMMA
+// issuer.  TMEM: S/P of tile i at [128i, 128i + 128), O of tile i at
+// [256 + D*i, 256 + D*i + D).  Tensor pipe order per key tile g (counted
+// across the CTA's items): PV0(g), S0(g+1), PV1(g), S1(g+1); S_i(g+1)
+// overwrites the P_i(g) columns PV_i(g) reads and is issued after it by the
+// same thread (UMMAs from one thread execute in order).  The first PV of an
+// item overwrites O, so the issuer waits until the softmax warps have read
+// the previous item's O out of TMEM (o_free).
+//
+// Barrier phases are counted per use across items; every wait is bounded
+// (2 s of %globaltimer, then the device status word and a CTA abort flag).
+#include <cmath>
+
+#include "isa_internal.h"
+#include "tc_ptx.cuh"
+
+namespace isa {
+
+namespace {
+
+template <int D>
+struct FusedCfg {
+  static constexpr int TILE = 128;
+  static constexpr int BN = 128;
+  static constexpr int Q_BYTES = TILE * D * 2;   // one 128-row tile
+  static constexpr int KT_BYTES = BN * D * 2;    // one key (or value) tile
+  static constexpr int OFF_Q = 0;                // [buffer][tile]
+  static constexpr int OFF_K = 4 * Q_BYTES;      // K hi, K lo
+  static constexpr int OFF_V = OFF_K + 2 * KT_BYTES;
+  static constexpr int OFF_BIAS = OFF_V + KT_BYTES;  // [2][BN] log2 cnt of key tiles g (ring by g & 1)
+  static constexpr int OFF_BAR = OFF_BIAS + 2 * BN * 4;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
+  static constexpr int THREADS = 320;
+  static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+struct FusedBars {
+  uint64_t q_full[2][2];  // [buffer][tile]
+  uint64_t q_empty[2];    // buffer free: last S of its item done
+  uint64_t k_full, v_full, k_empty, v_empty;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t o_free[2];     // O of tile i read out by its softmax warps
+  uint64_t teardown;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(FusedBars) <= 256, "barrier block");
+
+__device__ __forceinline__ void fraise(FusedBars* bars, const FlashParams& p) {
+  *reinterpret_cast<volatile int*>(&bars->abort) = 1;
+  if (p.status != nullptr) atomicCAS(p.status, 0, 5 /* ISA_ERR_DEVICE_TIMEOUT */);
+}
+__device__ __forceinline__ bool fw1(uint64_t* bar, uint32_t par, FusedBars* bars, const FlashParams& p) {
+  const int r = mbar_wait_bounded(bar, par, reinterpret_cast<volatile int*>(&bars->abort), kWaitLimitNs);
+  if (r == 2) fraise(bars, p);
+  return r == 0;
+}
+__device__ __forceinline__ bool fwarp(uint64_t* bar, uint32_t par, FusedBars* bars, const FlashParams& p) {
+  const bool ok = fw1(bar, par, bars, p);
+  return __all_sync(0xffffffffu, ok);
+}
+template <int N>
+__device__ __forceinline__ void fregs_after(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKhi,
+                 const __grid_constant__ CUtensorMap tmKlo, const __grid_constant__ CUtensorMap tmV,
+                 const FlashParams p, int n_items) {
+  using C = FusedCfg<D>;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  FusedBars* bars = reinterpret_cast<FusedBars*>(smem + C::OFF_BAR);
+  const uint32_t aQ = smem_u32(smem + C::OFF_Q);
+  const uint32_t aK = smem_u32(smem + C::OFF_K);
+  const uint32_t aV = smem_u32(smem + C::OFF_V);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = static_cast<int>(gridDim.x);
+  const int my_items = n_items > static_cast<int>(blockIdx.x) ? (n_items - 1 - static_cast<int>(blockIdx.x)) / G + 1 : 0;
+  const int nT = p.n_kv_tiles;
+  const int total = my_items * nT;  // key tiles this CTA walks, over all its items
+  auto item_of = [&](int k) { return static_cast<int>(blockIdx.x) + k * G; };
+
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->q_full[b][0], 1);
+      mbar_init(&bars->q_full[b][1], 1);
+      mbar_init(&bars->q_empty[b], 1);
+    }
+    mbar_init(&bars->k_full, 1);
+    mbar_init(&bars->v_full, 1);
+    mbar_init(&bars->k_empty, 1);
+    mbar_init(&bars->v_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_done[i], 1);
+      mbar_init(&bars->o_free[i], 128);
+    }
+    mbar_init(&bars->teardown, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmKhi);
+    tma_prefetch_desc(&tmKlo);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      int q_issued = 0, g_issued = 0;
+      auto load_q = [&](int k) -> bool {
+        const int b = k & 1;
+        if (k >= 2 && !fw1(&bars->q_empty[b], ((k >> 1) - 1) & 1, bars, p)) return false;
+        const int item = item_of(k);
+        const int bh = item / p.pairs_per_head, row0 = (item % p.pairs_per_head) * 256;
+        for (int i = 0; i < 2; ++i) {
+          mbar_arrive_expect_tx(&bars->q_full[b][i], C::Q_BYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(smem + C::OFF_Q + (b * 2 + i) * C::Q_BYTES + c * (128 * 128), &tmQ, &bars->q_full[b][i],
+                        c * 64, bh * p.N + row0 + i * 128);
+        }
+        q_issued = k + 1;
+        return true;
+      };
+      if (my_items > 0) ok = load_q(0);
+      for (int g = 0; ok && g < total; ++g) {
+        const int k = g / nT, t = g % nT;
+        const int bh = item_of(k) / p.pairs_per_head;
+        const int r = bh * p.kv_rows_per_head + t * BN;
+        if (g >= 1 && !(ok = fw1(&bars->k_empty, (g - 1) & 1, bars, p))) break;
+        mbar_arrive_expect_tx(&bars->k_full, 2 * C::KT_BYTES + BN * 4);
+        // key biases of tile g: slot g & 1 (the softmax of tile g-1 reads the
+        // other slot; it is done with slot g & 1 once S_1(g-1) has completed)
+        bulk_load(smem + C::OFF_BIAS + (g & 1) * BN * 4, p.bias2 + static_cast<size_t>(r), BN * 4, &bars->k_full);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(smem + C::OFF_K + c * (BN * 128), &tmKhi, &bars->k_full, c * 64, r);
+          tma_load_2d(smem + C::OFF_K + C::KT_BYTES + c * (BN * 128), &tmKlo, &bars->k_full, c * 64, r);
+        }
+        if (g >= 1 && !(ok = fw1(&bars->v_empty, (g - 1) & 1, bars, p))) break;
+        mbar_arrive_expect_tx(&bars->v_full, C::KT_BYTES);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) tma_load_2d(smem + C::OFF_V + c * (BN * 128), &tmV, &bars->v_full, c * 64, r);
+        g_issued = g + 1;
+        // the next item's Q, as soon as its buffer is free (during this item)
+        if (t == 0 && k + 1 < my_items && !(ok = load_q(k + 1))) break;
+      }
+      // drain own copies still in flight
+      if (g_issued > 0) {
+        mbar_wait_bounded(&bars->k_full, (g_issued - 1) & 1, nullptr, kWaitLimitNs);
+        mbar_wait_bounded(&bars->v_full, (g_issued - 1) & 1, nullptr, kWaitLimitNs);
+      }
+      for (int k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k) {
+        mbar_wait_bounded(&bars->q_full[k & 1][0], (k >> 1) & 1, nullptr, kWaitLimitNs);
+        mbar_wait_bounded(&bars->q_full[k & 1][1], (k >> 1) & 1, nullptr, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDS = idesc_bf16(128, BN, 0);
+      constexpr uint32_t IDO = idesc_bf16(128, D, 1);
+      bool ok = true;
+      // S_i(g) = Q_i (hi + lo) of key tile g; commits s_full[i]
+      auto issue_S = [&](int i, int g) {
+        const int k = g / nT;
+        const uint32_t qa = aQ + ((k & 1) * 2 + i) * C::Q_BYTES;
+        const uint32_t dS = tmem + i * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                    desc_k_sw128(aK + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                    desc_k_sw128(aK + C::KT_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, 1u);
+        umma_commit(&bars->s_full[i]);
+      };
+      // waits for the Q of key tile g's item (first tile of an item only)
+      auto q_ready = [&](int g) -> bool {
+        if (g % nT != 0) return true;
+        const int k = g / nT;
+        return fw1(&bars->q_full[k & 1][0], (k >> 1) & 1, bars, p) &&
+               fw1(&bars->q_full[k & 1][1], (k >> 1) & 1, bars, p);
+      };
+      auto issue_PV = [&](int i, int g) -> bool {
+        const int k = g / nT, t = g % nT;
+        if (t == 0 && k > 0 && !fw1(&bars->o_free[i], (k - 1) & 1, bars, p)) return false;
+        if (!fw1(&bars->p_full[i], g & 1, bars, p)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_tmem_a(tmem + 2 * BN + i * D, tmem + i * BN + kk * 8, desc_mn_sw128(aV + kk * 16 * 128, BN * 128),
+                           IDO, (t > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bars->o_done[i]);
+        return true;
+      };
+      if (total > 0) {
+        ok = q_ready(0) && fw1(&bars->k_full, 0, bars, p);
+        if (ok) {
+          tc_fence_after();
+          issue_S(0, 0);
+          issue_S(1, 0);
+          umma_commit(&bars->k_empty);
+          if (nT == 1) umma_commit(&bars->q_empty[0]);
+        }
+      }
+      for (int g = 0; ok && g < total; ++g) {
+        const bool more = g + 1 < total;
+        if (!(ok = fw1(&bars->v_full, g & 1, bars, p))) break;
+        if (!(ok = issue_PV(0, g))) break;
+        if (more) {
+          if (!(ok = q_ready(g + 1) && fw1(&bars->k_full, (g + 1) & 1, bars, p))) break;
+          tc_fence_after();
+          issue_S(0, g + 1);
+        }
+        if (!(ok = issue_PV(1, g))) break;
+        umma_commit(&bars->v_empty);
+        if (more) {
+          issue_S(1, g + 1);
+          umma_commit(&bars->k_empty);
+          // the item's last QK^T is issued: its Q buffer frees when it completes
+          if ((g + 1) % nT == nT - 1) umma_commit(&bars->q_empty[((g + 1) / nT) & 1]);
+        }
+      }
+      umma_commit(&bars->teardown);
+      mbar_wait_bounded(&bars->teardown, 0, nullptr, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------ softmax warpgroup of tile i
+    const int i = warp >> 2;
+    const int r = tid & 127;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t sS = tmem + lane_base + i * BN;
+    const uint32_t sO = tmem + lane_base + 2 * BN + i * D;
+    bool ok = true;
+    if (p.inject != nullptr && (__ldg(p.inject) & 1)) {  // test hook: behave as if S never arrived
+      fraise(bars, p);
+      ok = false;
+    }
+    for (int k = 0; ok && k < my_items; ++k) {
+      const int item = item_of(k);
+      const int bh = item / p.pairs_per_head;
+      const int g_row = (item % p.pairs_per_head) * 256 + i * 128 + r;  // query row in the head
+      float m = -INFINITY, l = 0.f, mx = -INFINITY;
+      for (int t = 0; t < nT; ++t) {
+        const int g = k * nT + t;
+        if (!(ok = fwarp(&bars->s_full[i], g & 1, bars, p))) break;
+        tc_fence_after();
+        const float* bias = reinterpret_cast<const float*>(smem + C::OFF_BIAS + (g & 1) * BN * 4);
+        // logits of half h (64 columns), in log2 units: s*log2(e)*S + log2 cnt
+        auto load_half = [&](int h, float (&x)[64]) {
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            uint32_t u[32];
+            tmem_ld32(sS + h * 64 + q2 * 32, u);
+            tmem_wait_ld();
+            fregs_after(u);
+            const float4* bp = reinterpret_cast<const float4*>(bias + h * 64 + q2 * 32);
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+              const float4 b = bp[c4];
+              const int c = 4 * c4;
+              x[q2 * 32 + c + 0] = fmaf(__uint_as_float(u[c + 0]), p.scale_log2, b.x);
+              x[q2 * 32 + c + 1] = fmaf(__uint_as_float(u[c + 1]), p.scale_log2, b.y);
+              x[q2 * 32 + c + 2] = fmaf(__uint_as_float(u[c + 2]), p.scale_log2, b.z);
+              x[q2 * 32 + c + 3] = fmaf(__uint_as_float(u[c + 3]), p.scale_log2, b.w);
+            }
+          }
+        };
+        float mt = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < BN / 64; ++h) {
+          float x[64];
+          load_half(h, x);
+          float pm[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) pm[c] = x[c];
+#pragma unroll
+          for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
+          mt = fmaxf(mt, fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))));
+        }
+        mx = fmaxf(mx, mt);
+        const float m_new = fmaxf(m, mt);
+        // rescale only when the running maximum grew by more than 2^32 (every
+        // p stays <= 2^32; exact after the final 1/l)
+        const bool need = m_new > m + 32.0f;
+        const float alpha = need ? ex2(m - m_new) : 1.f;
+        if (need) {
+          l *= alpha;
+          m = m_new;
+        }
+        const float mref = (m == -INFINITY) ? 0.f : m;
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < BN / 64; ++h) {
+          float x[64];
+          load_half(h, x);  // S columns [64h, 64h+64); P of half h goes to columns [32h, 32h+32)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            uint32_t w[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float e0 = ex2(x[j * 32 + 2 * c] - mref);
+              const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
+              ps[(2 * c) & 7] += e0;
+              ps[(2 * c + 1) & 7] += e1;
+              w[c] = pack_bf16(e0, e1);
+            }
+            tmem_st16(sS + h * 32 + j * 16, w);
+          }
+        }
+        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        // O_i rescale (PV_i(g-1) is complete, PV_i(g) not yet issued)
+        if (t > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int j = 0; j < D / 32; ++j) {
+            uint32_t u[32];
+            tmem_ld32(sO + j * 32, u);
+            tmem_wait_ld();
+            fregs_after(u);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+            tmem_st32(sO + j * 32, u);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[i]);
+      }
+      if (!ok) break;
+      // epilogue of item k: sharpness and Taylor output of this row
+      if (!(ok = fwarp(&bars->o_done[i], (k * nT + nT - 1) & 1, bars, p))) break;
+      tc_fence_after();
+      const bool store = g_row < p.n_rows;
+      uint16_t* orow = p.out + (static_cast<size_t>(bh) * p.N + (store ? g_row : 0)) * D;
+      const float inv = 1.f / l;
+      if (store) p.sharp[static_cast<size_t>(bh) * p.N + g_row] = ex2(mx - m) * inv;  // max_b softmax_b
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        uint32_t u[32];
+        tmem_ld32(sO + j * 32, u);
+        tmem_wait_ld();
+        fregs_after(u);
+        if (j == D / 32 - 1) {
+          // O of this tile is in registers: the next item's first PV may overwrite it
+          tc_fence_before();
+          mbar_arrive(&bars->o_free[i]);
+        }
+        if (store) {
+          uint4* o4 = reinterpret_cast<uint4*>(orow + j * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v4;
+            v4.x = pack_bf16(__uint_as_float(u[8 * q4 + 0]) * inv, __uint_as_float(u[8 * q4 + 1]) * inv);
+            v4.y = pack_bf16(__uint_as_float(u[8 * q4 + 2]) * inv, __uint_as_float(u[8 * q4 + 3]) * inv);
+            v4.z = pack_bf16(__uint_as_float(u[8 * q4 + 4]) * inv, __uint_as_float(u[8 * q4 + 5]) * inv);
+            v4.w = pack_bf16(__uint_as_float(u[8 * q4 + 6]) * inv, __uint_as_float(u[8 * q4 + 7]) * inv);
+            o4[q4] = v4;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi, const CUtensorMap& tmKlo,
+                         const CUtensorMap& tmV, const FlashParams& p0, int BH, cudaStream_t st) {
+  if (p0.n_rows <= 0 || BH <= 0 || p0.n_kv_tiles <= 0) return cudaSuccess;
+  FlashParams p = p0;
+  p.pairs_per_head = (p.n_rows + 255) / 256;
+  const long long items = static_cast<long long>(BH) * p.pairs_per_head;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  int dev = 0, nsm = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = static_cast<int>(items < nsm ? items : nsm);
+  if (D == 128) {
+    using C = FusedCfg<128>;
+    if ((e = cudaFuncSetAttribute(fused_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) !=
+        cudaSuccess)
+      return e;
+    fused_kernel<128><<<grid, C::THREADS, C::SMEM, st>>>(tmQ, tmKhi, tmKlo, tmV, p, static_cast<int>(items));
+  } else if (D == 64) {
+    using C = FusedCfg<64>;
+    const int smem = C::SMEM < 116 * 1024 ? 116 * 1024 : C::SMEM;  // one CTA per SM (all 512 TMEM columns)
+    if ((e = cudaFuncSetAttribute(fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+      return e;
+    fused_kernel<64><<<grid, C::THREADS, smem, st>>>(tmQ, tmKhi, tmKlo, tmV, p, static_cast<int>(items));
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace isa

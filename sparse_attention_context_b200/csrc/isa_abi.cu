@@ -248,7 +248,7 @@ int run_route_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, int32
   p.n_kv_tiles = d.nKpad / 128;
   p.kv_rows_per_head = d.nKpad;
   p.bias2 = at<float>(c.ws, c.L.bias2);
-  cudaError_t e = launch_attn2(d.d, 128, MODE_FUSED, tmQ, tmHi, tmLo, tmVb, p, d.BH, c.st);
+  cudaError_t e = launch_fused(d.d, tmQ, tmHi, tmLo, tmVb, p, d.BH, c.st);
   if (e == cudaSuccess) e = launch_route(sharp, routed, taylor, d.BH, d.N, d.n_route, c.status(), c.st);
   return cuda_status(e);
 }

@@ -62,6 +62,11 @@ cudaError_t launch_flash(int D, int BN, int mode, const CUtensorMap& tmK, const 
 // Two-tile engine (flash2.cu): DENSE, FULL and FUSED modes; grid
 // (ceil(n_rows/256), BH).  tmQ is read in DENSE / FUSED (contiguous rows,
 // box 64 x 128); tmK2 (the lo part of the split block means) only in FUSED.
+// Persistent sharpness + Taylor kernel (fused.cu): one CTA per SM looping
+// over 256-row items; tmQ over [BH*N, D] (box 128 rows), tmKhi / tmKlo / tmV
+// over the gathered kept operands [BH*kv_rows_per_head, D] (box 128 rows).
+cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi, const CUtensorMap& tmKlo,
+                         const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st);
 cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                          const CUtensorMap& tmK2, const CUtensorMap& tmV, const FlashParams& p, int BH,
                          cudaStream_t st);
