@@ -17,8 +17,10 @@
 // key tiles per item, a CTA per item spends most of its life loading Q from
 // HBM and storing O, one CTA per SM.  Here one CTA per SM loops over items
 // (stride = grid size): Q of the next item is loaded into a second buffer
-// while the current item computes, and the epilogue (O from TMEM to HBM) of
-// one item overlaps the QK^T products of the next.
+// while the current item computes, and the epilogue of one item overlaps the
+// QK^T products of the next: O goes from TMEM through registers into the
+// item's own Q buffer (free once its last QK^T is done) and leaves with one
+// TMA store per tile, so the softmax threads never wait on global stores.
 //
 // Warps (320 threads): 0-3 softmax of tile 0, 4-7 tile 1 (thread <-> query
 // row <-> TMEM lane), 8 TMA producer, 9 TMEM allocator + the single UMMA
@@ -60,7 +62,8 @@ struct FusedCfg {
 
 struct FusedBars {
   uint64_t q_full[2][2];  // [buffer][tile]
-  uint64_t q_empty[2];    // buffer free: last S of its item done
+  uint64_t q_empty[2];    // buffer free: its O tiles stored out of it (one arrival per tile)
+  uint64_t o_staged[2];   // O of tile i written into the staging buffer (128 arrivals)
   uint64_t k_full, v_full, k_empty, v_empty;
   uint64_t s_full[2];
   uint64_t p_full[2];
@@ -97,7 +100,7 @@ template <int D>
 __global__ void __launch_bounds__(320, 1)
     fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKhi,
                  const __grid_constant__ CUtensorMap tmKlo, const __grid_constant__ CUtensorMap tmV,
-                 const FlashParams p, int n_items) {
+                 const __grid_constant__ CUtensorMap tmO, const FlashParams p, int n_items) {
   using C = FusedCfg<D>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(320, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->q_full[b][0], 1);
       mbar_init(&bars->q_full[b][1], 1);
-      mbar_init(&bars->q_empty[b], 1);
+      mbar_init(&bars->q_empty[b], 2);
     }
     mbar_init(&bars->k_full, 1);
     mbar_init(&bars->v_full, 1);
@@ -130,6 +133,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bars->p_full[i], 128);
       mbar_init(&bars->o_done[i], 1);
       mbar_init(&bars->o_free[i], 128);
+      mbar_init(&bars->o_staged[i], 128);
     }
     mbar_init(&bars->teardown, 1);
     bars->abort = 0;
@@ -144,6 +148,7 @@ __global__ void __launch_bounds__(320, 1)
     tma_prefetch_desc(&tmKhi);
     tma_prefetch_desc(&tmKlo);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -250,7 +255,6 @@ __global__ void __launch_bounds__(320, 1)
           issue_S(0, 0);
           issue_S(1, 0);
           umma_commit(&bars->k_empty);
-          if (nT == 1) umma_commit(&bars->q_empty[0]);
         }
       }
       for (int g = 0; ok && g < total; ++g) {
@@ -267,8 +271,6 @@ __global__ void __launch_bounds__(320, 1)
         if (more) {
           issue_S(1, g + 1);
           umma_commit(&bars->k_empty);
-          // the item's last QK^T is issued: its Q buffer frees when it completes
-          if ((g + 1) % nT == nT - 1) umma_commit(&bars->q_empty[((g + 1) / nT) & 1]);
         }
       }
       umma_commit(&bars->teardown);
@@ -378,13 +380,17 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(&bars->p_full[i]);
       }
       if (!ok) break;
-      // epilogue of item k: sharpness and Taylor output of this row
+      // epilogue of item k: sharpness and Taylor output of this row.  O_i
+      // leaves TMEM through registers into Q buffer k & 1 (its last QK^T,
+      // S_1 of the item's last key tile, completed before PV_0 of that tile
+      // did, hence before o_done) in the TMA box layout, and one thread of
+      // the warpgroup stores the tile; rows past N are clipped by the map.
       if (!(ok = fwarp(&bars->o_done[i], (k * nT + nT - 1) & 1, bars, p))) break;
       tc_fence_after();
-      const bool store = g_row < p.n_rows;
-      uint16_t* orow = p.out + (static_cast<size_t>(bh) * p.N + (store ? g_row : 0)) * D;
+      const int b = k & 1;
+      uint8_t* stage = smem + C::OFF_Q + (b * 2 + i) * C::Q_BYTES;
       const float inv = 1.f / l;
-      if (store) p.sharp[static_cast<size_t>(bh) * p.N + g_row] = ex2(mx - m) * inv;  // max_b softmax_b
+      if (g_row < p.n_rows) p.sharp[static_cast<size_t>(bh) * p.N + g_row] = ex2(mx - m) * inv;  // max_b softmax_b
 #pragma unroll
       for (int j = 0; j < D / 32; ++j) {
         uint32_t u[32];
@@ -396,20 +402,34 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_before();
           mbar_arrive(&bars->o_free[i]);
         }
-        if (store) {
-          uint4* o4 = reinterpret_cast<uint4*>(orow + j * 32);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 v4;
-            v4.x = pack_bf16(__uint_as_float(u[8 * q4 + 0]) * inv, __uint_as_float(u[8 * q4 + 1]) * inv);
-            v4.y = pack_bf16(__uint_as_float(u[8 * q4 + 2]) * inv, __uint_as_float(u[8 * q4 + 3]) * inv);
-            v4.z = pack_bf16(__uint_as_float(u[8 * q4 + 4]) * inv, __uint_as_float(u[8 * q4 + 5]) * inv);
-            v4.w = pack_bf16(__uint_as_float(u[8 * q4 + 6]) * inv, __uint_as_float(u[8 * q4 + 7]) * inv);
-            o4[q4] = v4;
-          }
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t x = pack_bf16(__uint_as_float(u[8 * q4 + 0]) * inv, __uint_as_float(u[8 * q4 + 1]) * inv);
+          const uint32_t y = pack_bf16(__uint_as_float(u[8 * q4 + 2]) * inv, __uint_as_float(u[8 * q4 + 3]) * inv);
+          const uint32_t z = pack_bf16(__uint_as_float(u[8 * q4 + 4]) * inv, __uint_as_float(u[8 * q4 + 5]) * inv);
+          const uint32_t w = pack_bf16(__uint_as_float(u[8 * q4 + 6]) * inv, __uint_as_float(u[8 * q4 + 7]) * inv);
+          // 16-byte chunk (j*4 + q4) of the row: 64-column box j/2, chunk (j%2)*4 + q4 of its 128-byte row
+          st_shared_v4(smem_u32(stage) + (j >> 1) * (128 * 128) + sw128(r, (j & 1) * 4 + q4), x, y, z, w);
         }
       }
+      fence_proxy_async_smem();  // the generic-proxy writes above, for the TMA store
+      mbar_arrive(&bars->o_staged[i]);
+      if ((warp & 3) == 0 && lane == 0) {
+        if (fw1(&bars->o_staged[i], k & 1, bars, p)) {
+          const int row0 = (item % p.pairs_per_head) * 256 + i * 128;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) tma_store_3d(&tmO, stage + c * (128 * 128), c * 64, row0, bh);
+          bulk_commit_group();
+          bulk_wait_read_all();  // the staging buffer may be reloaded with Q once read
+          mbar_arrive(&bars->q_empty[b]);
+        } else {
+          ok = false;
+        }
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
     }
+    if ((warp & 3) == 0 && lane == 0) bulk_wait_all();  // stores complete before the CTA ends
   }
 
   tc_fence_before();
@@ -421,7 +441,8 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi, const CUtensorMap& tmKlo,
-                         const CUtensorMap& tmV, const FlashParams& p0, int BH, cudaStream_t st) {
+                         const CUtensorMap& tmV, const CUtensorMap& tmO, const FlashParams& p0, int BH,
+                         cudaStream_t st) {
   if (p0.n_rows <= 0 || BH <= 0 || p0.n_kv_tiles <= 0) return cudaSuccess;
   FlashParams p = p0;
   p.pairs_per_head = (p.n_rows + 255) / 256;
@@ -437,14 +458,14 @@ cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi
     if ((e = cudaFuncSetAttribute(fused_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) !=
         cudaSuccess)
       return e;
-    fused_kernel<128><<<grid, C::THREADS, C::SMEM, st>>>(tmQ, tmKhi, tmKlo, tmV, p, static_cast<int>(items));
+    fused_kernel<128><<<grid, C::THREADS, C::SMEM, st>>>(tmQ, tmKhi, tmKlo, tmV, tmO, p, static_cast<int>(items));
   } else if (D == 64) {
     using C = FusedCfg<64>;
     const int smem = C::SMEM < 116 * 1024 ? 116 * 1024 : C::SMEM;  // one CTA per SM (all 512 TMEM columns)
     if ((e = cudaFuncSetAttribute(fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return e;
-    fused_kernel<64><<<grid, C::THREADS, smem, st>>>(tmQ, tmKhi, tmKlo, tmV, p, static_cast<int>(items));
+    fused_kernel<64><<<grid, C::THREADS, smem, st>>>(tmQ, tmKhi, tmKlo, tmV, tmO, p, static_cast<int>(items));
   } else {
     return cudaErrorInvalidValue;
   }

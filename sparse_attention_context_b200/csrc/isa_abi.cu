@@ -231,9 +231,10 @@ int run_route_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, int32
   const Dims& d = c.d;
   int rc = run_build_kept(c, kept);
   if (rc != ISA_OK) return rc;
-  CUtensorMap tmQ, tmHi, tmLo, tmVb;
+  CUtensorMap tmQ, tmHi, tmLo, tmVb, tmO;
   const uint64_t kv_rows = static_cast<uint64_t>(d.BH) * d.nKpad;
   if (!make_tmap_bf16(&tmQ, q, static_cast<uint64_t>(d.BH) * d.N, d.d, 128) ||
+      !make_tmap_bf16_3d(&tmO, out, d.BH, d.N, d.d, 128) ||
       !make_tmap_bf16(&tmHi, at<uint16_t>(c.ws, c.L.Khi), kv_rows, d.d, 128) ||
       !make_tmap_bf16(&tmLo, at<uint16_t>(c.ws, c.L.Klo), kv_rows, d.d, 128) ||
       !make_tmap_bf16(&tmVb, at<uint16_t>(c.ws, c.L.Vb), kv_rows, d.d, 128))
@@ -248,7 +249,7 @@ int run_route_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, int32
   p.n_kv_tiles = d.nKpad / 128;
   p.kv_rows_per_head = d.nKpad;
   p.bias2 = at<float>(c.ws, c.L.bias2);
-  cudaError_t e = launch_fused(d.d, tmQ, tmHi, tmLo, tmVb, p, d.BH, c.st);
+  cudaError_t e = launch_fused(d.d, tmQ, tmHi, tmLo, tmVb, tmO, p, d.BH, c.st);
   if (e == cudaSuccess) e = launch_route(sharp, routed, taylor, d.BH, d.N, d.n_route, c.status(), c.st);
   return cuda_status(e);
 }
@@ -336,6 +337,18 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, int D, in
   const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1u, 1u};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int BH, int N, int D, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -52,6 +52,9 @@ struct FlashParams {
 // Bytes per CTA of key-split partials for head dim D.
 inline size_t split_bytes_per_cta(int D) { return 256ull * (static_cast<size_t>(D) * 4 + 8); }
 
+// Tensor map over [BH, N, D] bf16 (D innermost), box = 64 columns x box_rows
+// rows x 1 matrix, 128-byte swizzle: rows past N of a matrix are clipped.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, int BH, int N, int D, int box_rows);
 // Tensor map over a [rows, D] bf16 row-major matrix, box = 64 columns x
 // box_rows rows, 128-byte swizzle.  Returns false if encoding fails.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows);
@@ -64,9 +67,11 @@ cudaError_t launch_flash(int D, int BN, int mode, const CUtensorMap& tmK, const 
 // box 64 x 128); tmK2 (the lo part of the split block means) only in FUSED.
 // Persistent sharpness + Taylor kernel (fused.cu): one CTA per SM looping
 // over 256-row items; tmQ over [BH*N, D] (box 128 rows), tmKhi / tmKlo / tmV
-// over the gathered kept operands [BH*kv_rows_per_head, D] (box 128 rows).
+// over the gathered kept operands [BH*kv_rows_per_head, D] (box 128 rows),
+// tmO the 3-D map of out (make_tmap_bf16_3d, box 128 rows).
 cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi, const CUtensorMap& tmKlo,
-                         const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st);
+                         const CUtensorMap& tmV, const CUtensorMap& tmO, const FlashParams& p, int BH,
+                         cudaStream_t st);
 cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                          const CUtensorMap& tmK2, const CUtensorMap& tmV, const FlashParams& p, int BH,
                          cudaStream_t st);
