@@ -15,12 +15,8 @@
 //   FULL   ISA full attention for routed queries: gathered Q rows, keys of
 //          every source block then of the kept context blocks, one block
 //          per key tile, partial blocks masked by their token count.
-//   FUSED  ISA sharpness and 0-th order Taylor attention in one pass over
-//          every query: logits s*q.Kbar_b + log cnt_b from bf16 q times
-//          Kbar split into bf16 hi + lo parts (two UMMAs, fp32-grade), the
-//          block-mean values as V.  Writes the sharpness of every query and
-//          the Taylor output of every row (routed rows are overwritten by
-//          the FULL pass afterwards).
+// (Sharpness + Taylor over every query runs in the persistent kernel of
+// fused.cu, built on the same pipeline.)
 //
 // Work items: 256 query rows of one (b, h); whole waves of items run as
 // one launch, the items of a partial last wave are split along the key
@@ -53,15 +49,14 @@ namespace isa {
 template <int D, int BN, int MODE>
 struct Attn2Cfg {
   static constexpr int TILE = 128;
-  static constexpr bool kFused = MODE == MODE_FUSED;
   static constexpr bool kTmaQ = MODE != MODE_FULL;  // contiguous query rows
   static constexpr int Q_BYTES = TILE * D * 2;      // one tile
   static constexpr int KT_BYTES = BN * D * 2;       // one key (or value) tile
-  static constexpr int NKT = kFused ? 3 : 2;        // tiles per stage: K[,Klo],V
+  static constexpr int NKT = 2;                     // tiles per stage: K, V
   // P hand-off in parts of 64 keys (one barrier each), so PV starts on the
   // first keys while the softmax still exponentiates the rest (32-key parts
-  // measured no faster: twice the issuer's waits); FUSED hands P over whole.
-  static constexpr int NP = kFused ? 1 : BN / 64;
+  // measured no faster: twice the issuer's waits).
+  static constexpr int NP = BN / 64;
   static constexpr int STAGE_BYTES = NKT * KT_BYTES;
   static constexpr int BUDGET = 225 * 1024;
   static constexpr int ST_FIT = (BUDGET - 2 * Q_BYTES - 1024 - 256) / STAGE_BYTES;
@@ -69,7 +64,7 @@ struct Attn2Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + STAGES * STAGE_BYTES;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + runtime key-bias table (FUSED)
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
   static constexpr int THREADS = 320;
   static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
   static_assert(ST_FIT >= 1, "shared memory budget");
@@ -136,7 +131,7 @@ __device__ __forceinline__ int kv_count(const FlashParams& p, int bh, int t) {
 template <int D, int BN, int MODE>
 __global__ void __launch_bounds__(320, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmK2, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmV,
                  const FlashParams p) {
   using C = Attn2Cfg<D, BN, MODE>;
   constexpr int ST = C::STAGES;
@@ -182,7 +177,6 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 8 && lane == 0) {
     if constexpr (C::kTmaQ) tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
-    if constexpr (C::kFused) tma_prefetch_desc(&tmK2);
     tma_prefetch_desc(&tmV);
   }
   tc_fence_before();
@@ -210,14 +204,9 @@ __global__ void __launch_bounds__(320, 1)
         if (t >= ST && !w1(&bars->k_empty[st], ((t / ST) - 1) & 1, bars, p)) break;
         const int r = kv_row<BN, MODE>(p, bh, kv0 + t);
         uint8_t* base = smem + C::OFF_KV + st * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&bars->k_full[st], (C::kFused ? 2 : 1) * C::KT_BYTES);
+        mbar_arrive_expect_tx(&bars->k_full[st], C::KT_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) tma_load_2d(base + c * (BN * 128), &tmK, &bars->k_full[st], c * 64, r);
-        if constexpr (C::kFused) {
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(base + C::KT_BYTES + c * (BN * 128), &tmK2, &bars->k_full[st], c * 64, r);
-        }
         uint8_t* vb = base + (C::NKT - 1) * C::KT_BYTES;
         if (t >= ST && !w1(&bars->v_empty[st], ((t / ST) - 1) & 1, bars, p)) break;
         mbar_arrive_expect_tx(&bars->v_full[st], C::KT_BYTES);
@@ -252,12 +241,6 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < D / 16; ++kk)
           umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
                     desc_k_sw128(kb + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, kk > 0 ? 1u : 0u);
-        if constexpr (C::kFused) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
-                      desc_k_sw128(kb + C::KT_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, 1u);
-        }
         umma_commit(&bars->s_full[i]);
       };
       // PV_i(t), part by part as the softmax hands P over (false: a wait gave up)
@@ -363,83 +346,21 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t sS = tmem + lane_base + i * BN;
     const uint32_t sO = tmem + lane_base + 2 * BN + i * D;
-    float m = -INFINITY, l = 0.f, mx = -INFINITY;
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
     if (p.inject != nullptr && (__ldg(p.inject) & 1)) {  // test hook: behave as if S never arrived
       raise2(bars, p);
       ok = false;
     }
-    // FUSED: the head's log2(cnt) key biases (-inf padding) in shared memory.
-    float* sBias = reinterpret_cast<float*>(smem + C::OFF_BAR + 256);
-    if constexpr (C::kFused) {
-      for (int c = tid; c < p.kv_rows_per_head; c += 256)
-        sBias[c] = __ldg(p.bias2 + static_cast<size_t>(bh) * p.kv_rows_per_head + c);
-      asm volatile("bar.sync 1, 256;" ::: "memory");  // the two softmax warpgroups only
-    }
-    // Softmax on 64-column halves of the S tile (a second tcgen05.ld of S
-    // replaces keeping all BN logits in registers: 10 warps per SM leave
-    // 168 registers per thread).
-    constexpr int NH = BN / 64;
     int valid_next = nT > 0 ? kv_count<BN, MODE>(p, bh, kv0) : 0;
     for (int t = 0; ok && t < nT; ++t) {
       const int valid = valid_next;
       if (t + 1 < nT) valid_next = kv_count<BN, MODE>(p, bh, kv0 + t + 1);  // prefetched under the wait below
       if (!(ok = wwarp(&bars->s_full[i], t & 1, bars, p))) break;
       tc_fence_after();
-      uint32_t sreg[C::kFused ? 1 : BN / 32][32];
-      const float* bias = C::kFused ? sBias + (kv0 + t) * BN : nullptr;
-      // logits of half h, in log2 units (-inf outside the tile's tokens)
-      auto load_half = [&](int h, float (&x)[64]) {
-        if constexpr (C::kFused) {
-          // 32 columns at a time: the bias reads stay out of the TMEM registers' way
-#pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            uint32_t u[32];
-            tmem_ld32(sS + h * 64 + q2 * 32, u);
-            tmem_wait_ld();
-            regs_after(u);
-            const float4* bp = reinterpret_cast<const float4*>(bias + h * 64 + q2 * 32);
-#pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4) {
-              const float4 b = bp[c4];
-              const int c = 4 * c4;
-              x[q2 * 32 + c + 0] = fmaf(__uint_as_float(u[c + 0]), p.scale_log2, b.x);
-              x[q2 * 32 + c + 1] = fmaf(__uint_as_float(u[c + 1]), p.scale_log2, b.y);
-              x[q2 * 32 + c + 2] = fmaf(__uint_as_float(u[c + 2]), p.scale_log2, b.z);
-              x[q2 * 32 + c + 3] = fmaf(__uint_as_float(u[c + 3]), p.scale_log2, b.w);
-            }
-          }
-        } else {
-          uint32_t u[2][32];
-          tmem_ld32(sS + h * 64, u[0]);
-          tmem_ld32(sS + h * 64 + 32, u[1]);
-          tmem_wait_ld();
-          regs_after(u[0]);
-          regs_after(u[1]);
-#pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(u[c >> 5][c & 31]) * p.scale_log2;
-          if (valid < (h + 1) * 64) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (h * 64 + c >= valid) x[c] = -INFINITY;
-          }
-        }
-      };
+      uint32_t sreg[BN / 32][32];
       float mt = -INFINITY;
-      if constexpr (C::kFused) {
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          float x[64];
-          load_half(h, x);
-          float pm[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) pm[k] = x[k];
-#pragma unroll
-          for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
-          mt = fmaxf(mt, fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))));
-        }
-      } else {
+      {
         // every S column of the tile in flight at once; max of the raw
         // scores (the scale is positive), columns past `valid` excluded.
         // The scores stay in registers for the exponent pass below.
@@ -465,7 +386,6 @@ __global__ void __launch_bounds__(320, 1)
                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         mt = raw * p.scale_log2;
       }
-      mx = fmaxf(mx, mt);
       const float m_new = fmaxf(m, mt);
       // Rescale only when the running maximum grew by more than 2^32: with
       // the stale reference every p stays <= 2^32 (bf16 and fp32 hold that
@@ -483,26 +403,7 @@ __global__ void __launch_bounds__(320, 1)
       const float mref = (m == -INFINITY) ? 0.f : m;
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      if constexpr (C::kFused) {
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          float x[64];
-          load_half(h, x);  // S columns [64h, 64h+64); P of half h goes to columns [32h, 32h+32)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            uint32_t w[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float e0 = ex2(x[j * 32 + 2 * c] - mref);
-              const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
-              ps[(2 * c) & 7] += e0;
-              ps[(2 * c + 1) & 7] += e1;
-              w[c] = pack_bf16(e0, e1);
-            }
-            tmem_st16(sS + h * 32 + j * 16, w);
-          }
-        }
-      } else {
+      {
         // quarters of 32 columns; P of quarter q goes to columns [16q, 16q+16)
         // (the scores are already in registers)
         const float nm = -mref;
@@ -565,30 +466,9 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_before();
         mbar_arrive(&bars->p_part[i][BN / 64 - 1]);
       }
-      if constexpr (!C::kFused) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) ps[k] += ps2[k].x + ps2[k].y;
-      }
+      for (int k = 0; k < 4; ++k) ps[k] += ps2[k].x + ps2[k].y;
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      if constexpr (C::kFused) {
-        // O_i rescale (PV_i(t-1) is complete, PV_i(t) not yet issued), done
-        // after the logits left the registers; then P goes over whole
-        if (t > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-          for (int j = 0; j < D / 32; ++j) {
-            uint32_t u[32];
-            tmem_ld32(sO + j * 32, u);
-            tmem_wait_ld();
-            regs_after(u);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
-            tmem_st32(sO + j * 32, u);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_part[i][0]);
-      }
     }
 
     const bool valid_row = g < p.n_rows;
@@ -597,10 +477,6 @@ __global__ void __launch_bounds__(320, 1)
       int dst = valid_row ? (p.row_idx ? __ldg(p.row_idx + static_cast<size_t>(bh) * p.n_rows + g) : g) : 0;
       const bool store = valid_row && static_cast<unsigned>(dst) < static_cast<unsigned>(p.N);
       if (!store) dst = 0;
-      if constexpr (C::kFused) {
-        // sharpness = max_b softmax_b = 2^(mx - m) / l (l is relative to m)
-        if (store) p.sharp[static_cast<size_t>(bh) * p.N + dst] = ex2(mx - m) / l;
-      }
       if (split) {
         // unnormalised partial accumulator of this key range (+ its m, l)
         const size_t prow = static_cast<size_t>(blockIdx.x) * 256 + i * 128 + r;
@@ -694,11 +570,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }
 
 template <int D, int BN, int MODE>
-static cudaError_t launch2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmK2,
+static cudaError_t launch2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const FlashParams& p0, int BH, cudaStream_t st) {
   using C = Attn2Cfg<D, BN, MODE>;
   auto kern = attn2_kernel<D, BN, MODE>;
-  int smem = C::SMEM + (C::kFused ? p0.kv_rows_per_head * 4 : 0);  // + FUSED key biases
+  int smem = C::SMEM;
   if (smem < 116 * 1024) smem = 116 * 1024;                         // one CTA per SM (all 512 TMEM columns)
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -716,7 +592,7 @@ static cudaError_t launch2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK, con
   const long long whole = nsm > 0 ? items / nsm * nsm : items;
   const int rem = static_cast<int>(items - whole);
   int pieces = 0;
-  if (!C::kFused && rem > 0 && p.o_part != nullptr && p.split_capacity > 0) {
+  if (rem > 0 && p.o_part != nullptr && p.split_capacity > 0) {
     pieces = nsm / rem;
     if (pieces > p.n_kv_tiles / 4) pieces = p.n_kv_tiles / 4;
     while (pieces > 1 && pieces * rem > p.split_capacity) --pieces;
@@ -724,14 +600,14 @@ static cudaError_t launch2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK, con
   }
   const long long first = pieces ? whole : items;
   if (first > 0) {
-    kern<<<static_cast<unsigned>(first), C::THREADS, smem, st>>>(tmQ, tmK, tmK2, tmV, p);
+    kern<<<static_cast<unsigned>(first), C::THREADS, smem, st>>>(tmQ, tmK, tmV, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (pieces) {
     FlashParams ps = p;
     ps.item_base = static_cast<int>(whole);
     ps.split_pieces = pieces;
-    kern<<<static_cast<unsigned>(rem * pieces), C::THREADS, smem, st>>>(tmQ, tmK, tmK2, tmV, ps);
+    kern<<<static_cast<unsigned>(rem * pieces), C::THREADS, smem, st>>>(tmQ, tmK, tmV, ps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     combine_kernel<D><<<(rem * 256 + 7) / 8, 256, 0, st>>>(p.o_part, p.ml_part, pieces, static_cast<int>(whole), rem,
                                                            p);
@@ -741,19 +617,17 @@ static cudaError_t launch2_t(const CUtensorMap& tmQ, const CUtensorMap& tmK, con
 }
 
 cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                         const CUtensorMap& tmK2, const CUtensorMap& tmV, const FlashParams& p, int BH,
+                         const CUtensorMap& tmV, const FlashParams& p, int BH,
                          cudaStream_t st) {
   if (p.n_rows <= 0 || BH <= 0) return cudaSuccess;
 #define ISA_ATTN2_CASE(d_, bn_, m_) \
-  if (D == d_ && BN == bn_ && mode == m_) return launch2_t<d_, bn_, m_>(tmQ, tmK, tmK2, tmV, p, BH, st);
+  if (D == d_ && BN == bn_ && mode == m_) return launch2_t<d_, bn_, m_>(tmQ, tmK, tmV, p, BH, st);
   ISA_ATTN2_CASE(128, 128, MODE_DENSE)
   ISA_ATTN2_CASE(128, 128, MODE_FULL)
   ISA_ATTN2_CASE(128, 64, MODE_FULL)
-  ISA_ATTN2_CASE(128, 128, MODE_FUSED)
   ISA_ATTN2_CASE(64, 128, MODE_DENSE)
   ISA_ATTN2_CASE(64, 128, MODE_FULL)
   ISA_ATTN2_CASE(64, 64, MODE_FULL)
-  ISA_ATTN2_CASE(64, 128, MODE_FUSED)
 #undef ISA_ATTN2_CASE
   return cudaErrorInvalidValue;
 }

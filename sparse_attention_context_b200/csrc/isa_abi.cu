@@ -271,7 +271,7 @@ int run_full(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t*
     p.kept_ctx = kept;
     p.n_kv_tiles = d.nSB + d.n_keep;
     p.kv_rows_per_head = d.N;
-    e = launch_attn2(d.d, d.blk, MODE_FULL, tmK /* Q is gathered by threads */, tmK, tmK, tmV, p, d.BH, c.st);
+    e = launch_attn2(d.d, d.blk, MODE_FULL, tmK /* Q is gathered by threads */, tmK, tmV, p, d.BH, c.st);
   }
   return cuda_status(e);
 }
@@ -503,7 +503,7 @@ int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* 
     p.ml_part = at<float2>(ws, align256(kCtlBytes + static_cast<size_t>(cap) * 256 * d * 4));
     p.split_capacity = cap;
   }
-  return cuda_status(launch_attn2(d, 128, MODE_DENSE, tmQ, tmK, tmK, tmV, p, static_cast<int>(BH),
+  return cuda_status(launch_attn2(d, 128, MODE_DENSE, tmQ, tmK, tmV, p, static_cast<int>(BH),
                                   static_cast<cudaStream_t>(stream)));
 }
 

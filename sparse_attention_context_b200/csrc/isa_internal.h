@@ -15,7 +15,7 @@ constexpr int kTopkCap = 4096;     // max context blocks the top-k sort holds
 constexpr int kSalRows = 32;       // query blocks per saliency CTA
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
-enum FlashMode { MODE_DENSE = 0, MODE_FULL = 1, MODE_TAYLOR = 2, MODE_SHARP = 3, MODE_FUSED = 4 };
+enum FlashMode { MODE_DENSE = 0, MODE_FULL = 1, MODE_TAYLOR = 2, MODE_SHARP = 3 };
 
 // Arguments of the tcgen05 attention engine (one CTA = 128 query rows of
 // one (b, h); grid = (ceil(n_rows/128), B*H)).
@@ -62,9 +62,9 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, int D, in
 // One-tile engine (flash.cu): SHARP and TAYLOR modes; grid (ceil(n_rows/128), BH).
 cudaError_t launch_flash(int D, int BN, int mode, const CUtensorMap& tmK, const CUtensorMap& tmV,
                          const FlashParams& p, int BH, cudaStream_t st);
-// Two-tile engine (flash2.cu): DENSE, FULL and FUSED modes; grid
-// (ceil(n_rows/256), BH).  tmQ is read in DENSE / FUSED (contiguous rows,
-// box 64 x 128); tmK2 (the lo part of the split block means) only in FUSED.
+// Two-tile engine (flash2.cu): DENSE and FULL modes; 256-row work items,
+// whole waves in one launch plus a key-split tail and its merge.  tmQ is
+// read in DENSE (contiguous rows, box 64 x 128); FULL gathers Q by threads.
 // Persistent sharpness + Taylor kernel (fused.cu): one CTA per SM looping
 // over 256-row items; tmQ over [BH*N, D] (box 128 rows), tmKhi / tmKlo / tmV
 // over the gathered kept operands [BH*kv_rows_per_head, D] (box 128 rows),
@@ -73,8 +73,7 @@ cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi
                          const CUtensorMap& tmV, const CUtensorMap& tmO, const FlashParams& p, int BH,
                          cudaStream_t st);
 cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                         const CUtensorMap& tmK2, const CUtensorMap& tmV, const FlashParams& p, int BH,
-                         cudaStream_t st);
+                         const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st);
 
 // Stage-1 kernels.
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,
