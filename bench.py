@@ -65,10 +65,10 @@ def counts(cfg):
 # source, or another workload, the report's traffic is null.
 FULL_TRAFFIC = {
     "config": "480p",
-    "bytes": 387_516_672 + 37_400_064 + 15_112_960 + 11_520 + 18_467_328,
+    "bytes": 394_686_208 + 38_460_160 + 15_115_520 + 7_936 + 18_466_816,
     "sources": {
-        "sparse_attention_context_b200/csrc/flash2.cu": "6e65216d95f4e63af94970034b00c2b978e01593ead2f49c1bc3fb718ca7f816",
-        "sparse_attention_context_b200/csrc/tc_ptx.cuh": "014a3c466b7859b30d53c5e121984b9e032b9ddec01309fde00c3151e40b0a26",
+        "sparse_attention_context_b200/csrc/flash2.cu": "fb5f09457eb0885f74352c7ab5bfbec9d8d196fe7c2876f729bbb09329e52598",
+        "sparse_attention_context_b200/csrc/tc_ptx.cuh": "a99eac8f56d3542436ffd184ac1c8e2e863e048d2eef2dcbc2189b53b0161f21",
     },
 }
 
