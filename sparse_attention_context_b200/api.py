@@ -143,31 +143,88 @@ def isa_taylor_attn_fwd(q, kept, taylor, shape: IsaShape, ws, out, stream=None):
 
 
 def isa_forward(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, ws=None, out=None,
-                stream=None):
+                stream=None, groups=None):
     """All ISA stages in one call.
 
     CUDA inputs: runs on the current stream and returns a CUDA tensor.
     CPU inputs (the host-buffer path): copies q, k, v to the GPU, runs, and
-    copies the output back into a pinned CPU tensor (returned).
+    copies the output back into a pinned CPU tensor (returned).  Every
+    (b, h) is an independent unit, so the heads are taken in `groups`
+    consecutive slices (default: 4 when there are at least 8 heads): the
+    host-to-device copy of a slice, the forward of the previous slice and the
+    device-to-host copy of the one before run on three streams at once, and
+    PCIe transfers in both directions overlap the GPU work.  Pass pinned
+    host tensors for the copies to be asynchronous.
     """
-    host = not q.is_cuda
-    if host:
-        dev = torch.device("cuda")
-        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
-    shape = make_shape(q, N_src, block, keep, rho, scale)
-    if ws is None:
-        ws = new_workspace(shape, q.device)
-    o = torch.empty_like(q) if (out is None or host) else out
-    _check_qkv(q, k, v, o)
-    rc = lib().isa_forward(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                           ws.data_ptr(), ws.numel(), _stream(stream))
-    check("isa_forward", rc)
-    if host:
-        dst = out if out is not None else torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        dst.copy_(o, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        return dst
-    return o
+    if q.is_cuda:
+        shape = make_shape(q, N_src, block, keep, rho, scale)
+        if ws is None:
+            ws = new_workspace(shape, q.device)
+        o = torch.empty_like(q) if out is None else out
+        _check_qkv(q, k, v, o)
+        rc = lib().isa_forward(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                               ws.data_ptr(), ws.numel(), _stream(stream))
+        check("isa_forward", rc)
+        return o
+    return _isa_forward_host(q, k, v, N_src, block, keep, rho, scale, ws, out, groups)
+
+
+def _isa_forward_host(q, k, v, N_src, block, keep, rho, scale, ws, out, groups):
+    """Host-buffer path of isa_forward: head slices pipelined over a copy-in
+    stream, the caller's current stream (compute) and a copy-out stream."""
+    dev = torch.device("cuda")
+    B, H, N, d = q.shape
+    BH = B * H
+    G = groups if groups is not None else (4 if BH >= 8 else 1)
+    G = max(1, min(int(G), BH))
+    bounds = [BH * i // G for i in range(G + 1)]
+    qf, kf, vf = (t.reshape(BH, N, d) for t in (q, k, v))
+    dq, dk, dv = (torch.empty((BH, N, d), dtype=q.dtype, device=dev) for _ in range(3))
+    do = torch.empty((BH, N, d), dtype=q.dtype, device=dev)
+    dst = out if out is not None else torch.empty((B, H, N, d), dtype=q.dtype, pin_memory=True)
+    dstf = dst.reshape(BH, N, d)
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    start = torch.cuda.Event()
+    start.record(comp)
+    s_in.wait_event(start)
+    s_out.wait_event(start)
+    big = max(bounds[i + 1] - bounds[i] for i in range(G))
+    shape_big = make_shape(torch.empty((1, big, N, d), device="meta"), N_src, block, keep, rho, scale)
+    if ws is None or ws.numel() < lib().isa_workspace_size(ctypes.byref(shape_big)):
+        ws = new_workspace(shape_big, dev)
+    done_in, done_comp = [], []
+    for g in range(G):
+        a, b = bounds[g], bounds[g + 1]
+        with torch.cuda.stream(s_in):
+            for src, buf in ((qf, dq), (kf, dk), (vf, dv)):
+                buf[a:b].copy_(src[a:b], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s_in)
+            done_in.append(ev)
+    for g in range(G):
+        a, b = bounds[g], bounds[g + 1]
+        comp.wait_event(done_in[g])
+        shape = make_shape(torch.empty((1, b - a, N, d), device="meta"), N_src, block, keep, rho, scale)
+        rc = lib().isa_forward(ctypes.byref(shape), dq[a].data_ptr(), dk[a].data_ptr(), dv[a].data_ptr(),
+                               do[a].data_ptr(), ws.data_ptr(), ws.numel(), _stream(None))
+        check("isa_forward", rc)
+        ev = torch.cuda.Event()
+        ev.record(comp)
+        done_comp.append(ev)
+    with torch.cuda.stream(s_out):
+        for g in range(G):
+            a, b = bounds[g], bounds[g + 1]
+            s_out.wait_event(done_comp[g])
+            dstf[a:b].copy_(do[a:b], non_blocking=True)
+    fin = torch.cuda.Event()
+    fin.record(s_out)
+    comp.wait_event(fin)
+    comp.synchronize()
+    for t in (dq, dk, dv, do, ws):  # keep the caching allocator from reusing them early
+        t.record_stream(s_in)
+        t.record_stream(s_out)
+    return dst
 
 
 def isa_forward_static(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, out=None,

@@ -80,3 +80,21 @@ def test_isa_full_size_sampled(cuda_ok, name, heads):
             rng.choice(routed, min(96, nr), replace=False), rng.choice(taylor, 96, replace=False),
             [0, cfg.N_src - 1, cfg.N_src, cfg.N - 1]]))
         compare_head(cfg.replace(H=H), bits, g, 0, h, cfg.keep, cfg.rho, rows=rows)
+
+
+@pytest.mark.parametrize("groups", [1, 5, None])
+def test_host_buffer_path(cuda_ok, groups):
+    """isa_forward on pinned host tensors (the end-to-end path: head slices
+    pipelined over copy-in, compute and copy-out streams) gives the device
+    path's output: index sets are per head, so only the key-split merge of
+    the full-attention tail (which depends on how many heads share a launch)
+    may round differently."""
+    cfg = CONFIGS["small"]
+    bits, (q, k, v) = inputs(cfg)
+    ref = api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    got = api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, groups=groups)
+    assert not got.is_cuda and got.shape == q.shape
+    check_out(got.double().numpy(), ref.double().cpu().numpy(), f"host path, groups={groups}")
+    if groups == 1:
+        assert torch.equal(got.view(torch.int16), ref.cpu().view(torch.int16))  # same launches: same bits
