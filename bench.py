@@ -251,6 +251,52 @@ def run_reference(args, cfg):
     print(json.dumps(rec), flush=True)
 
 
+def run_sweep(args):
+    """Latency of the ISA forward over the keep x rho grid of the sweep
+    workload (B=1, H=24, d=128, 32768 + 32768 tokens, block 128) beside the
+    in-house dense kernel; one JSON line per grid point.  The oracle error of
+    every grid point is checked by tests/test_gpu_sweep.py."""
+    import torch
+
+    from sparse_attention_context_b200 import api
+
+    cfg = CONFIGS["sweep"]
+    if args.heads:
+        cfg = cfg.replace(H=args.heads)
+    q, k, v = (to_torch_bf16(b).cuda() for b in make_inputs(cfg, seed=0))
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, warm, n):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    dws = api.dense_workspace(cfg.d)
+    dout = torch.empty_like(q)
+    dense_ms = timed(lambda: api.isa_dense_attn_fwd(q, k, v, out=dout, ws=dws), 1, 2)
+    del dout
+    dense_flops = 4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d
+    out = torch.empty_like(q)
+    for keep in (0.1, 0.25, 0.5, 1.0):
+        for rho in (0.0, 0.1, 0.2, 0.5, 1.0):
+            shape = api.make_shape(q, cfg.N_src, cfg.block, keep, rho)
+            ws = api.new_workspace(shape)
+            ms = timed(lambda: api.isa_forward(q, k, v, cfg.N_src, cfg.block, keep, rho, ws=ws, out=out),
+                       max(args.warmup, 1), max(args.steps, 1))
+            assert api.isa_read_device_status(ws) == 0
+            print(json.dumps({"sweep": cfg.name, "H": cfg.H, "keep": keep, "rho": rho, "ms": round(ms, 4),
+                              "dense_ms": round(dense_ms, 3), "isa_over_dense": round(ms / dense_ms, 4),
+                              "eff_tflops": round(dense_flops / (ms * 1e-3) / 1e12, 1)}), flush=True)
+            del ws
+
+
 def config_dict(cfg, n):
     return {"workload": f"ISA fwd {cfg.name}-latent: B={cfg.B} H={cfg.H} d={cfg.d} N_src={cfg.N_src} "
                         f"N_ctx={cfg.N_ctx} block={cfg.block} keep={cfg.keep} rho={cfg.rho}",
@@ -272,7 +318,11 @@ def main():
     ap.add_argument("--heads", type=int, default=None, help="override H (small profiling captures)")
     ap.add_argument("--rho", type=float, default=None, help="override rho (profiling captures)")
     ap.add_argument("--keep", type=float, default=None, help="override keep (profiling captures)")
+    ap.add_argument("--sweep", action="store_true", help="keep x rho latency grid of the sweep workload")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     cfg = CONFIGS[args.config]
     if args.heads:
         cfg = cfg.replace(H=args.heads)

@@ -91,7 +91,8 @@ def compare_head(cfg: Config, bits, g, b, h, keep, rho, rows=None):
     q, k, v = (bf16_bits_to_f64(x[b, h]) for x in bits)
     H = bits[0].shape[1]
     bh = b * H + h
-    ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, keep, rho)
+    # the sets are decided on all rows either way; `rows` only limits the outputs
+    ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, keep, rho, rows=rows)
     # stage 1
     if g["sal"] is not None and ref["nCB"] > 0:
         s_gpu = g["sal"].reshape(-1, ref["nCB"])[bh]
@@ -100,7 +101,7 @@ def compare_head(cfg: Config, bits, g, b, h, keep, rho, rows=None):
     same_kept = check_set(kept_gpu, ref["kept_ctx"], ref["sal_ctx"], ref["n_keep"])
     assert np.all(np.diff(kept_gpu) > 0), "kept not ascending"
     if not same_kept:
-        ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, keep, rho, kept_override=kept_gpu)
+        ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, keep, rho, kept_override=kept_gpu, rows=rows)
     # stage 2
     sh_gpu = g["sharp"].reshape(-1, cfg.N)[bh]
     assert np.allclose(sh_gpu, ref["sharp"], rtol=1e-4, atol=1e-7), \
