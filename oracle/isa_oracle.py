@@ -32,7 +32,11 @@ The exact formulas below are the plainest reading of that outline:
 * 0-th order Taylor attention: exp(s q.k_j) is replaced by exp(s q.Kbar_b)
   for every j in block b, in numerator and denominator; summing over the
   block turns this into attention over block means with an additive ln cnt_b
-  bias and block-mean values.
+  bias and block-mean values;
+* variant grouping by whole query blocks (``granularity="block"``): a query
+  block (same per-segment partition as the keys) scores the mean sharpness
+  of its queries, and the n_route_blocks = ceil(rho*nB - 1e-6*nB) best
+  blocks (ties: lower block index) are routed whole.
 
 Pins (see tests/test_oracle_pins.py): the saliency and sharpness formulas are
 readings, not printed by the pages ("parity unpinned" as to the pages); they
@@ -161,6 +165,32 @@ def sharpness(q, Kbar_K, cnt_K, scale):
 
 
 # ---------------------------------------------------------------------------
+# Variant of the grouping step: whole query blocks.  The abstract names a
+# dynamic grouping of queries but not the unit that is grouped; this variant
+# groups at the granularity of the token blocks already used for the keys,
+# so that a routed group is a run of consecutive query rows.
+# ---------------------------------------------------------------------------
+
+def n_route_blocks_of(rho: float, nB: int) -> int:
+    """Number of query blocks routed to full attention: ceil(rho*nB - 1e-6*nB) in [0, nB]."""
+    return int(min(max(math.ceil(rho * nB - 1e-6 * nB), 0), nB))
+
+
+def block_mean_sharpness(sharp, starts, cnts):
+    """Score of every query block: the mean sharpness of its cnt_b queries."""
+    return np.array([sharp[s:s + c].sum() / c for s, c in zip(starts, cnts)], dtype=np.float64)
+
+
+def route_query_blocks(sharp, starts, cnts, rho):
+    """Block-granular grouping: the n_route_blocks query blocks of highest
+    mean sharpness (ties: lower block index first) are routed whole.
+    Returns (block scores, n_route_blocks, routed block indices ascending)."""
+    score = block_mean_sharpness(sharp, starts, cnts)
+    nrb = n_route_blocks_of(rho, len(starts))
+    return score, nrb, topk_ascending(score, nrb)
+
+
+# ---------------------------------------------------------------------------
 # Stage 3: full attention for routed queries
 # ---------------------------------------------------------------------------
 
@@ -196,14 +226,18 @@ def taylor_rows(q_rows, Kbar_K, Vbar_K, cnt_K, scale, chunk=4096):
 # ---------------------------------------------------------------------------
 
 def isa_head(q, k, v, N_src, blk, keep, rho, scale=None,
-             kept_override=None, routed_override=None, rows=None):
+             kept_override=None, routed_override=None, rows=None, granularity="token"):
     """ISA forward for one head, all stages in order; float64 inputs [N, d].
 
     ``kept_override`` / ``routed_override`` replace the selected context
     block set / routed query set (used to re-run the later stages on a set
-    that differs from the oracle's only inside the tie window).
+    that differs from the oracle's only inside the tie window); with
+    ``granularity="block"`` the routed override is a set of query blocks.
     ``rows`` restricts which output rows are computed (others are NaN);
     every stage that decides a set still runs on all rows.
+    ``granularity`` selects the dynamic query grouping: "token" routes the
+    n_route sharpest queries one by one; "block" routes whole query blocks
+    (see ``route_query_blocks``).
     Returns a dict of every intermediate and the output.
     """
     N, d = q.shape
@@ -222,8 +256,19 @@ def isa_head(q, k, v, N_src, blk, keep, rho, scale=None,
 
     Kb = kept_blocks(nSB, kept_ctx)
     sharp = sharpness(q, Kbar[Kb], cnts[Kb], s)
-    nr = n_route_of(rho, N)
-    routed = topk_ascending(sharp, nr) if routed_override is None else np.asarray(routed_override, dtype=np.int64)
+    extra = {}
+    if granularity == "token":
+        nr = n_route_of(rho, N)
+        routed = topk_ascending(sharp, nr) if routed_override is None else np.asarray(routed_override, dtype=np.int64)
+    elif granularity == "block":
+        score, nrb, rblocks = route_query_blocks(sharp, starts, cnts, rho)
+        if routed_override is not None:
+            rblocks = np.asarray(routed_override, dtype=np.int64)
+        routed = kept_tokens(starts, cnts, rblocks)
+        nr = len(routed)
+        extra = dict(block_score=score, n_route_blocks=nrb, routed_blocks=rblocks)
+    else:
+        raise ValueError(granularity)
     mask = np.ones(N, dtype=bool)
     mask[routed] = False
     taylor = np.nonzero(mask)[0].astype(np.int64)
@@ -240,7 +285,7 @@ def isa_head(q, k, v, N_src, blk, keep, rho, scale=None,
     return dict(out=out, Qbar=Qbar, Kbar=Kbar, Vbar=Vbar, cnts=cnts, nSB=nSB, nCB=nCB,
                 sal_all=sal_all, sal_ctx=sal_ctx, kept_ctx=kept_ctx, kept_blocks=Kb,
                 sharp=sharp, routed=routed, taylor=taylor, tokens=T,
-                n_keep=nk, n_route=nr, scale=s)
+                n_keep=nk, n_route=nr, scale=s, **extra)
 
 
 def isa_fwd(q, k, v, N_src, blk, keep, rho, scale=None):
