@@ -132,7 +132,7 @@ class ClockSampler:
                "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
                "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
-    def __init__(self, torch_device, period_s=0.005):
+    def __init__(self, torch_device, period_s=0.002):
         self.dev = torch_device
         self.period = period_s
         self.sm, self.mx, self.reasons, self.err = [], None, set(), None
@@ -297,6 +297,83 @@ def run_sweep(args):
             del ws
 
 
+def run_block_grouping(args):
+    """The block-granular grouping variant on the 480p latent workload beside
+    the per-token grouping: latency of both forwards (CUDA events), the
+    stage split of the block variant, and the approximation error of each
+    against full attention for every query over the same kept tokens
+    (rho = 1), Sum|o - o_full| / Sum|o_full|.  One JSON line.  Oracle parity
+    of the variant is checked by tests/test_gpu_block_route.py."""
+    import torch
+
+    from sparse_attention_context_b200 import api
+
+    cfg = CONFIGS[args.config]
+    if args.heads:
+        cfg = cfg.replace(H=args.heads)
+    if args.rho is not None:
+        cfg = cfg.replace(rho=args.rho)
+    if args.keep is not None:
+        cfg = cfg.replace(keep=args.keep)
+    q, k, v = (to_torch_bf16(b).cuda() for b in make_inputs(cfg, seed=0))
+    stream = torch.cuda.current_stream()
+    shape = api.make_shape(q, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    ws = api.new_workspace(shape)
+    out_t, out_b = torch.empty_like(q), torch.empty_like(q)
+
+    def timed(fn, warm, n):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    W, K = max(args.warmup, 3), max(args.steps, 1)
+    ms_tok = timed(lambda: api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws, out=out_t), W, K)
+    ms_blk = timed(lambda: api.isa_forward_blocks(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws,
+                                                  out=out_b), W, K)
+    # stage split of the block variant
+    kept = torch.empty((cfg.B, cfg.H, api.isa_n_keep(shape)), dtype=torch.int32, device=q.device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    acc = np.zeros(3)
+    for i in range(W + K):
+        ev[0].record(stream)
+        api.isa_preselect_ctx(q, k, v, shape, ws, kept=kept, want_saliency=False)
+        ev[1].record(stream)
+        _, rows, _, _ = api.isa_route_blocks_taylor_fwd(q, kept, shape, ws, out_b, want_scores=False,
+                                                        want_sharpness=False)
+        ev[2].record(stream)
+        api.isa_full_attn_rows_fwd(q, k, v, kept, rows, shape, ws, out_b)
+        ev[3].record(stream)
+        torch.cuda.synchronize()
+        if i >= W:
+            acc += [ev[j].elapsed_time(ev[j + 1]) for j in range(3)]
+    acc /= K
+    assert api.isa_read_device_status(ws) == 0
+    ref = api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, 1.0)  # every query on full attention
+    torch.cuda.synchronize()
+    ref_abs = ref.float().abs().sum().item()
+
+    def err(o):
+        d = (o.float() - ref.float()).abs()
+        return {"mean_rel": round(d.sum().item() / ref_abs, 6), "max_abs": round(d.max().item(), 5)}
+
+    nrb = api.isa_n_route_blocks(shape)
+    print(json.dumps({
+        "variant": "block-granular query grouping", "config": config_dict(cfg, 1),
+        "token_grouping_ms": round(ms_tok, 4), "block_grouping_ms": round(ms_blk, 4),
+        "block_stage_ms": {"preselect": round(acc[0], 4), "sharpness_taylor_route_blocks": round(acc[1], 4),
+                           "full_attn_rows": round(acc[2], 4)},
+        "routed_queries": {"token": api.isa_n_route(shape), "block_rows": nrb * cfg.block, "blocks": nrb},
+        "error_vs_full_over_kept": {"token": err(out_t), "block": err(out_b)},
+        "steps": K, "warmup": W}), flush=True)
+
+
 def config_dict(cfg, n):
     return {"workload": f"ISA fwd {cfg.name}-latent: B={cfg.B} H={cfg.H} d={cfg.d} N_src={cfg.N_src} "
                         f"N_ctx={cfg.N_ctx} block={cfg.block} keep={cfg.keep} rho={cfg.rho}",
@@ -319,9 +396,14 @@ def main():
     ap.add_argument("--rho", type=float, default=None, help="override rho (profiling captures)")
     ap.add_argument("--keep", type=float, default=None, help="override keep (profiling captures)")
     ap.add_argument("--sweep", action="store_true", help="keep x rho latency grid of the sweep workload")
+    ap.add_argument("--grouping", default="token", choices=["token", "block"],
+                    help="block: time the block-granular query grouping variant beside the per-token one")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.grouping == "block":
+        run_block_grouping(args)
         return
     cfg = CONFIGS[args.config]
     if args.heads:
@@ -399,6 +481,10 @@ def main():
         for i in range(args.steps):
             step(i)
         t1.record(stream)
+        # wait by polling (sleep releases the GIL) so the sampler thread runs
+        # while the GPU works; a blocking synchronize here starves it
+        while not t1.query():
+            time.sleep(2e-4)
         torch.cuda.synchronize()
     barrier()
     ms = t0.elapsed_time(t1) / args.steps

@@ -78,6 +78,11 @@ int isa_n_keep(const isa_shape* shape);
 /* Number of routed queries per (b, h): ceil(rho*N - 1e-6*N).  -1 if invalid. */
 int isa_n_route(const isa_shape* shape);
 
+/* Number of routed query blocks per (b, h) of the block-granular grouping
+ * (isa_route_blocks_taylor_fwd): ceil(rho*nB - 1e-6*nB), nB = nSB + nCB.
+ * -1 if invalid. */
+int isa_n_route_blocks(const isa_shape* shape);
+
 /* Bytes of workspace needed by every ISA call on this shape (0 if invalid). */
 size_t isa_workspace_size(const isa_shape* shape);
 
@@ -136,6 +141,44 @@ int isa_full_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t*
 int isa_taylor_attn_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
                         const int32_t* taylor_idx, uint16_t* out, void* ws, size_t ws_bytes,
                         void* stream);
+
+/* Stage 3 for an explicit row list: full attention, over every token of
+ * every source block and of the kept context blocks, for the n_rows entries
+ * of row_idx [B, H, n_rows] int32 per (b, h).  An entry of -1 is padding:
+ * it is computed on a zero query and never stored; any other entry outside
+ * [0, N) is skipped and reported as ISA_ERR_INVALID_ARG in the device
+ * status word.  Entries must not repeat within a (b, h).  With
+ * row_idx = routed_idx and n_rows = n_route this is isa_full_attn_fwd. */
+int isa_full_attn_rows_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const int32_t* kept_ctx_idx, const int32_t* row_idx, int n_rows, uint16_t* out,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Stages 2 and 4 with the dynamic query grouping taken over whole query
+ * blocks (a variant reading: the abstract does not fix the unit grouped).
+ * Query blocks use the per-segment partition of the keys; block b scores
+ * the mean sharpness of its cnt_b queries (fp32); the n_rb =
+ * isa_n_route_blocks() best blocks (ties: lower block index) are routed.
+ * Like isa_route_taylor_fwd, writes the 0-th order Taylor output of EVERY
+ * row of out; follow it with isa_full_attn_rows_fwd(routed_rows,
+ * n_rb * block) to overwrite the routed blocks' rows with full attention.
+ *   routed_blk_idx [B, H, n_rb] int32 out: routed block numbers (source
+ *                  blocks 0..nSB-1, then context blocks), ascending.
+ *   routed_rows    [B, H, n_rb * block] int32 out: entry r*block + t is
+ *                  row t of routed block r, or -1 past a partial block's
+ *                  last row.
+ *   block_score    [B, H, nB] float out (mean sharpness per block), or NULL.
+ *   sharpness      [B, H, N] float out, or NULL.
+ * Supported up to nB = 16384 query blocks per head (else
+ * ISA_ERR_UNSUPPORTED).  routed_* may be NULL when n_rb == 0. */
+int isa_route_blocks_taylor_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
+                                int32_t* routed_blk_idx, int32_t* routed_rows, float* block_score,
+                                float* sharpness, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/* The forward with block-granular grouping: isa_preselect_ctx,
+ * isa_route_blocks_taylor_fwd, isa_full_attn_rows_fwd on one stream, with
+ * every index set held inside ws.  out [B, H, N, d] bf16. */
+int isa_forward_blocks(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
 /* All four stages in order on one stream (isa_preselect_ctx,
  * isa_route_taylor_fwd, isa_full_attn_fwd), with the kept set and the

@@ -38,6 +38,7 @@ _SH = ctypes.POINTER(IsaShape)
 SIGNATURES = {
     "isa_n_keep": (_I, [_SH]),
     "isa_n_route": (_I, [_SH]),
+    "isa_n_route_blocks": (_I, [_SH]),
     "isa_workspace_size": (_SZ, [_SH]),
     "isa_preselect_ctx": (_I, [_SH, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_route_queries": (_I, [_SH, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -45,6 +46,9 @@ SIGNATURES = {
     "isa_route_taylor_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_full_attn_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_taylor_attn_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
+    "isa_full_attn_rows_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "isa_route_blocks_taylor_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "isa_forward_blocks": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_forward": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_forward_static": (_I, [_SH, _P, _P, _P, _P, _P]),
     "isa_dense_workspace_size": (_SZ, [_I]),

@@ -41,6 +41,10 @@ def isa_n_route(shape: IsaShape) -> int:
     return lib().isa_n_route(ctypes.byref(shape))
 
 
+def isa_n_route_blocks(shape: IsaShape) -> int:
+    return lib().isa_n_route_blocks(ctypes.byref(shape))
+
+
 def isa_workspace_size(shape: IsaShape) -> int:
     return lib().isa_workspace_size(ctypes.byref(shape))
 
@@ -140,6 +144,51 @@ def isa_taylor_attn_fwd(q, kept, taylor, shape: IsaShape, ws, out, stream=None):
                                    ws.numel(), _stream(stream))
     check("isa_taylor_attn_fwd", rc)
     return out
+
+
+def isa_full_attn_rows_fwd(q, k, v, kept, rows, shape: IsaShape, ws, out, stream=None):
+    """Stage 3 for an explicit row list rows [B,H,n_rows] (-1 entries are padding)."""
+    _check_qkv(q, k, v, out)
+    n_rows = rows.shape[-1]
+    rc = lib().isa_full_attn_rows_fwd(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                      _ptr(kept) if kept.numel() else None, _ptr(rows) if rows.numel() else None,
+                                      int(n_rows), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+    check("isa_full_attn_rows_fwd", rc)
+    return out
+
+
+def isa_route_blocks_taylor_fwd(q, kept, shape: IsaShape, ws, out, want_scores=True, want_sharpness=True,
+                                stream=None):
+    """Stages 2 + 4 with whole query blocks routed.  Returns (routed block
+    indices [B,H,n_rb], routed rows [B,H,n_rb*block] with -1 pads, block
+    scores [B,H,nB] or None, sharpness [B,H,N] or None)."""
+    _check_qkv(q, out)
+    B, H, N = shape.B, shape.H, shape.N_src + shape.N_ctx
+    nB = -(-shape.N_src // shape.block) + -(-shape.N_ctx // shape.block)
+    nrb = isa_n_route_blocks(shape)
+    rblk = torch.empty((B, H, nrb), dtype=torch.int32, device=q.device)
+    rows = torch.empty((B, H, nrb * shape.block), dtype=torch.int32, device=q.device)
+    score = torch.empty((B, H, nB), dtype=torch.float32, device=q.device) if want_scores else None
+    sharp = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if want_sharpness else None
+    rc = lib().isa_route_blocks_taylor_fwd(ctypes.byref(shape), q.data_ptr(), _ptr(kept) if kept.numel() else None,
+                                           _ptr(rblk) if nrb else None, _ptr(rows) if nrb else None, _ptr(score),
+                                           _ptr(sharp), out.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+    check("isa_route_blocks_taylor_fwd", rc)
+    return rblk, rows, score, sharp
+
+
+def isa_forward_blocks(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, ws=None,
+                       out=None, stream=None):
+    """The ISA forward with block-granular query grouping (CUDA tensors)."""
+    shape = make_shape(q, N_src, block, keep, rho, scale)
+    if ws is None:
+        ws = new_workspace(shape, q.device)
+    o = torch.empty_like(q) if out is None else out
+    _check_qkv(q, k, v, o)
+    rc = lib().isa_forward_blocks(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  ws.data_ptr(), ws.numel(), _stream(stream))
+    check("isa_forward_blocks", rc)
+    return o
 
 
 def isa_forward(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, ws=None, out=None,

@@ -14,7 +14,9 @@
 //   DENSE  all N keys, contiguous queries (the in-house baseline).
 //   FULL   ISA full attention for routed queries: gathered Q rows, keys of
 //          every source block then of the kept context blocks, one block
-//          per key tile, partial blocks masked by their token count.
+//          per key tile, partial blocks masked by their token count.  A row
+//          index of -1 is a padding entry (a partial block's missing rows
+//          in the block-granular grouping): computed on zeros, never stored.
 // (Sharpness + Taylor over every query runs in the persistent kernel of
 // fused.cu, built on the same pipeline.)
 //
@@ -328,7 +330,7 @@ __global__ void __launch_bounds__(320, 1)
           const int src = p.row_idx ? __ldg(p.row_idx + static_cast<size_t>(bh) * p.n_rows + gg) : gg;
           if (static_cast<unsigned>(src) < static_cast<unsigned>(p.N))
             vals[it] = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.N + src) * D + ch * 8));
-          else if (p.status != nullptr)
+          else if (src != -1 && p.status != nullptr)  // -1: a padding entry, skipped silently
             atomicCAS(p.status, 0, 1 /* ISA_ERR_INVALID_ARG: index out of range, row skipped */);
         }
       }
@@ -544,7 +546,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   if (g >= p.n_rows) return;
   int dst = p.row_idx ? __ldg(p.row_idx + static_cast<size_t>(bh) * p.n_rows + g) : g;
   if (static_cast<unsigned>(dst) >= static_cast<unsigned>(p.N)) {
-    if (lane == 0 && p.status != nullptr) atomicCAS(p.status, 0, 1);
+    if (dst != -1 && lane == 0 && p.status != nullptr) atomicCAS(p.status, 0, 1);  // -1: padding
     return;
   }
   float M = -INFINITY;

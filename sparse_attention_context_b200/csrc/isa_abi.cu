@@ -16,12 +16,13 @@ namespace isa {
 namespace {
 
 struct Dims {
-  int B, H, BH, N_src, N_ctx, N, d, blk, nSB, nCB, nB, n_keep, n_route, nK, nKpad, nChunks;
+  int B, H, BH, N_src, N_ctx, N, d, blk, nSB, nCB, nB, n_keep, n_route, n_rb, nK, nKpad, nChunks;
   float scale;
 };
 
 struct WsLayout {
-  size_t Qbar, Kbar, Vbar, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, opart, mlpart, total;
+  size_t Qbar, Kbar, Vbar, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, rblk, rrows, opart, mlpart,
+      total;
   int split_ctas;  // key-split partial CTAs the workspace holds
 };
 
@@ -74,6 +75,7 @@ int check_shape(const isa_shape* s, Dims* o) {
   d.nB = d.nSB + d.nCB;
   d.n_keep = keep_count(s->keep, d.nCB);
   d.n_route = route_count(s->rho, d.N);
+  d.n_rb = route_count(s->rho, d.nB);  // block-granular grouping: same rule over the nB query blocks
   d.nK = d.nSB + d.n_keep;
   d.nKpad = (d.nK + 127) / 128 * 128;
   d.nChunks = (d.nB + kSalRows - 1) / kSalRows;
@@ -104,6 +106,8 @@ WsLayout layout(const Dims& d) {
   L.kept = take(BH * std::max(d.n_keep, 1) * 4);
   L.routed = take(BH * std::max(d.n_route, 1) * 4);
   L.taylor = take(BH * std::max(d.N - d.n_route, 1) * 4);
+  L.rblk = take(BH * std::max(d.n_rb, 1) * 4);
+  L.rrows = take(BH * std::max(d.n_rb * d.blk, 1) * 4);
   L.split_ctas = split_ctas_for_device();
   L.opart = take(static_cast<size_t>(L.split_ctas) * 256 * d.d * 4);
   L.mlpart = take(static_cast<size_t>(L.split_ctas) * 256 * 8);
@@ -227,7 +231,7 @@ int run_route(const Ctx& c, const uint16_t* q, const int32_t* kept, int32_t* rou
 // Stages 2 and 4 in one pass over q: sharpness and the Taylor output of
 // every row (fused kernel), then routing.
 int run_route_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, int32_t* routed, int32_t* taylor,
-                     float* sharp_user, uint16_t* out) {
+                     float* sharp_user, uint16_t* out, bool route = true) {
   const Dims& d = c.d;
   int rc = run_build_kept(c, kept);
   if (rc != ISA_OK) return rc;
@@ -250,15 +254,17 @@ int run_route_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, int32
   p.kv_rows_per_head = d.nKpad;
   p.bias2 = at<float>(c.ws, c.L.bias2);
   cudaError_t e = launch_fused(d.d, tmQ, tmHi, tmLo, tmVb, tmO, p, d.BH, c.st);
-  if (e == cudaSuccess) e = launch_route(sharp, routed, taylor, d.BH, d.N, d.n_route, c.status(), c.st);
+  if (e == cudaSuccess && route) e = launch_route(sharp, routed, taylor, d.BH, d.N, d.n_route, c.status(), c.st);
   return cuda_status(e);
 }
 
-int run_full(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kept,
-             const int32_t* routed, uint16_t* out) {
+// Full attention for an explicit row list of n_rows entries per (b, h)
+// (entries of -1 are padding: computed on zeros, never stored).
+int run_full_rows(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kept,
+                  const int32_t* rows, int n_rows, uint16_t* out) {
   const Dims& d = c.d;
   cudaError_t e = cudaSuccess;
-  if (d.n_route > 0) {
+  if (n_rows > 0) {
     CUtensorMap tmK, tmV;
     if (!make_tmap_bf16(&tmK, k, static_cast<uint64_t>(d.BH) * d.N, d.d, d.blk) ||
         !make_tmap_bf16(&tmV, v, static_cast<uint64_t>(d.BH) * d.N, d.d, d.blk))
@@ -266,14 +272,31 @@ int run_full(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t*
     FlashParams p = base_params(c);
     p.q = q;
     p.out = out;
-    p.row_idx = routed;
-    p.n_rows = d.n_route;
+    p.row_idx = rows;
+    p.n_rows = n_rows;
     p.kept_ctx = kept;
     p.n_kv_tiles = d.nSB + d.n_keep;
     p.kv_rows_per_head = d.N;
     e = launch_attn2(d.d, d.blk, MODE_FULL, tmK /* Q is gathered by threads */, tmK, tmV, p, d.BH, c.st);
   }
   return cuda_status(e);
+}
+
+int run_full(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kept,
+             const int32_t* routed, uint16_t* out) {
+  return run_full_rows(c, q, k, v, kept, routed, c.d.n_route, out);
+}
+
+// Block-granular variant of run_route_taylor: the same fused sharpness +
+// Taylor pass over every row, then whole query blocks are routed.
+int run_route_blocks_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, int32_t* routed_blk,
+                            int32_t* routed_rows, float* score_user, float* sharp_user, uint16_t* out) {
+  const Dims& d = c.d;
+  float* sharp = sharp_user ? sharp_user : at<float>(c.ws, c.L.sharp);
+  int rc = run_route_taylor(c, q, kept, nullptr, nullptr, sharp, out, /*route=*/false);
+  if (rc != ISA_OK) return rc;
+  return cuda_status(launch_route_blocks(sharp, routed_blk, routed_rows, score_user, d.BH, d.N_src, d.N_ctx, d.blk,
+                                         d.n_rb, c.status(), c.st));
 }
 
 int run_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, const int32_t* taylor, uint16_t* out,
@@ -369,6 +392,11 @@ int isa_n_route(const isa_shape* shape) {
   return check_shape(shape, &d) == ISA_OK ? d.n_route : -1;
 }
 
+int isa_n_route_blocks(const isa_shape* shape) {
+  Dims d;
+  return check_shape(shape, &d) == ISA_OK ? d.n_rb : -1;
+}
+
 size_t isa_workspace_size(const isa_shape* shape) {
   Dims d;
   if (check_shape(shape, &d) != ISA_OK) return 0;
@@ -461,6 +489,51 @@ int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, co
   rc = run_preselect(c, q, k, v, kept, nullptr);
   if (rc == ISA_OK) rc = run_route_taylor(c, q, kept, routed, taylor, nullptr, out);
   if (rc == ISA_OK) rc = run_full(c, q, k, v, kept, routed, out);
+  return rc;
+}
+
+int isa_route_blocks_taylor_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
+                                int32_t* routed_blk_idx, int32_t* routed_rows, float* block_score, float* sharpness,
+                                uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (c.d.nB > kRouteBlocksCap) return ISA_ERR_UNSUPPORTED;
+  if (!tensors_ok({q, out})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_rb > 0 && !tensors_ok({routed_blk_idx, routed_rows})) return ISA_ERR_INVALID_ARG;
+  if ((block_score != nullptr && !aligned16(block_score)) || (sharpness != nullptr && !aligned16(sharpness)))
+    return ISA_ERR_INVALID_ARG;
+  return run_route_blocks_taylor(c, q, kept_ctx_idx, routed_blk_idx, routed_rows, block_score, sharpness, out);
+}
+
+int isa_full_attn_rows_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const int32_t* kept_ctx_idx, const int32_t* row_idx, int n_rows, uint16_t* out,
+                           void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (n_rows < 0) return ISA_ERR_INVALID_ARG;
+  if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (n_rows > 0 && (row_idx == nullptr || !aligned16(row_idx))) return ISA_ERR_INVALID_ARG;
+  if (static_cast<long long>(c.d.BH) * n_rows >= INT_MAX) return ISA_ERR_UNSUPPORTED;
+  return run_full_rows(c, q, k, v, kept_ctx_idx, row_idx, n_rows, out);
+}
+
+int isa_forward_blocks(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (c.d.nB > kRouteBlocksCap) return ISA_ERR_UNSUPPORTED;
+  if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
+  int32_t* kept = at<int32_t>(ws, c.L.kept);
+  int32_t* rblk = at<int32_t>(ws, c.L.rblk);
+  int32_t* rrows = at<int32_t>(ws, c.L.rrows);
+  rc = run_preselect(c, q, k, v, kept, nullptr);
+  if (rc == ISA_OK) rc = run_route_blocks_taylor(c, q, kept, rblk, rrows, nullptr, nullptr, out);
+  if (rc == ISA_OK) rc = run_full_rows(c, q, k, v, kept, rrows, c.d.n_rb * c.d.blk, out);
   return rc;
 }
 

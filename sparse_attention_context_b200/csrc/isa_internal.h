@@ -13,6 +13,7 @@ constexpr int kInjectOffset = 4;   // int32 fault-injection word (tests)
 constexpr int kCtlBytes = 256;
 constexpr int kTopkCap = 4096;     // max context blocks the top-k sort holds
 constexpr int kSalRows = 32;       // query blocks per saliency CTA
+constexpr int kRouteBlocksCap = 16384;  // max query blocks per head of the block grouping
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
 enum FlashMode { MODE_DENSE = 0, MODE_FULL = 1, MODE_TAYLOR = 2, MODE_SHARP = 3 };
@@ -87,5 +88,10 @@ cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_
                               int blk, int n_keep, int nKpad, int* status, cudaStream_t st);
 cudaError_t launch_route(const float* sharp, int32_t* routed, int32_t* taylor, int BH, int N, int n_route,
                          int* status, cudaStream_t st);
+// Block-granular grouping (route_blocks.cu): routed_blk [BH, n_rb] ascending
+// block indices, routed_rows [BH, n_rb*blk] rows of those blocks (-1 pads),
+// score_out [BH, nB] block mean sharpness or null.
+cudaError_t launch_route_blocks(const float* sharp, int32_t* routed_blk, int32_t* routed_rows, float* score_out,
+                                int BH, int N_src, int N_ctx, int blk, int n_rb, int* status, cudaStream_t st);
 
 }  // namespace isa

@@ -55,6 +55,8 @@ def test_counts_match_oracle(L, keep, rho, N_src, N_ctx, blk):
     nCB = -(-N_ctx // blk)
     assert L.isa_n_keep(ctypes.byref(s)) == oracle.n_keep_of(keep, nCB)
     assert L.isa_n_route(ctypes.byref(s)) == oracle.n_route_of(rho, N_src + N_ctx)
+    nB = -(-N_src // blk) + nCB
+    assert L.isa_n_route_blocks(ctypes.byref(s)) == oracle.n_route_blocks_of(rho, nB)
 
 
 def test_workspace_size(L):
@@ -92,6 +94,10 @@ def test_bad_pointers_and_workspace_rejected(L):
     assert L.isa_preselect_ctx(ctypes.byref(s), p, p, p, None, None, p, need, None) == 1       # kept missing
     assert L.isa_route_queries(ctypes.byref(s), p, p, None, p, None, p, need, None) == 1       # routed missing
     assert L.isa_attn_fwd(ctypes.byref(s), p, p, p, p, p, p, None, p, need, None) == 1         # out missing
+    assert L.isa_full_attn_rows_fwd(ctypes.byref(s), p, p, p, p, p, -1, p, p, need, None) == 1  # negative rows
+    assert L.isa_full_attn_rows_fwd(ctypes.byref(s), p, p, p, p, None, 4, p, p, need, None) == 1  # rows missing
+    assert L.isa_route_blocks_taylor_fwd(ctypes.byref(s), p, p, None, p, None, None, p, p, need, None) == 1
+    assert L.isa_forward_blocks(ctypes.byref(s), p, p, p, p, p, need - 1, None) == 3             # small ws
     assert L.isa_dense_attn_fwd(1, 1, 128, 80, 0.0, p, p, p, p, p, 256, None) == 2
     assert L.isa_dense_attn_fwd(1, 1, 128, 64, 0.0, p, p, p, p, p, 8, None) == 3
     assert L.isa_dense_attn_fwd(1, 1, 0, 64, 0.0, p, p, p, p, p, 256, None) == 1
