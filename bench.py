@@ -65,9 +65,9 @@ def counts(cfg):
 # source, or another workload, the report's traffic is null.
 FULL_TRAFFIC = {
     "config": "480p",
-    "bytes": 394_686_208 + 38_460_160 + 15_115_520 + 7_936 + 18_466_816,
+    "bytes": 384_441_088 + 36_827_392 + 14_966_272 + 768 + 18_468_864,
     "sources": {
-        "sparse_attention_context_b200/csrc/flash2.cu": "fb5f09457eb0885f74352c7ab5bfbec9d8d196fe7c2876f729bbb09329e52598",
+        "sparse_attention_context_b200/csrc/flash2.cu": "88a1e0b4f250bdc90e7b7e9834951c272f145ee77aabc0ae46734358e9a49539",
         "sparse_attention_context_b200/csrc/tc_ptx.cuh": "a99eac8f56d3542436ffd184ac1c8e2e863e048d2eef2dcbc2189b53b0161f21",
     },
 }
