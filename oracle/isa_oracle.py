@@ -33,6 +33,9 @@ The exact formulas below are the plainest reading of that outline:
   for every j in block b, in numerator and denominator; summing over the
   block turns this into attention over block means with an additive ln cnt_b
   bias and block-mean values;
+* variant stage 4 of first order (``taylor_order=1``): the linear term of
+  exp around the block mean is kept, which adds s * C_b^T q per kept block
+  to the numerator, C_b = sum_{j in b} (k_j - Kbar_b) v_j^T;
 * variant grouping by whole query blocks (``granularity="block"``): a query
   block (same per-segment partition as the keys) scores the mean sharpness
   of its queries, and the n_route_blocks = ceil(rho*nB - 1e-6*nB) best
@@ -222,11 +225,48 @@ def taylor_rows(q_rows, Kbar_K, Vbar_K, cnt_K, scale, chunk=4096):
 
 
 # ---------------------------------------------------------------------------
+# Variant of stage 4: first-order Taylor sparse attention.  The abstract's
+# "0-th order" names the first member of a family; the next member keeps
+# the linear term of exp around the block mean:
+#   e^{s q.k_j} ~= e^{s q.Kbar_b} (1 + s q.(k_j - Kbar_b))   for j in b.
+# In the denominator the linear terms of a block sum to zero (the deviations
+# from the block mean sum to zero), so it stays sum_b cnt_b e^{s q.Kbar_b};
+# the numerator gains s * C_b^T q per block, C_b = sum_{j in b} (k_j -
+# Kbar_b) v_j^T (a d x d matrix).
+# ---------------------------------------------------------------------------
+
+def correction_matrices(k, v, starts, cnts, blocks):
+    """C_b = sum_{j in b} (k_j - Kbar_b) v_j^T for the given blocks, float64 [n, d, d]."""
+    d = k.shape[1]
+    out = np.empty((len(blocks), d, d), dtype=np.float64)
+    for r, b in enumerate(blocks):
+        kb = k[starts[b]:starts[b] + cnts[b]]
+        vb = v[starts[b]:starts[b] + cnts[b]]
+        out[r] = (kb - kb.mean(axis=0)).T @ vb
+    return out
+
+
+def taylor1_rows(q_rows, Kbar_K, Vbar_K, C_K, cnt_K, scale, chunk=1024):
+    """o_i = [sum_b cnt_b e^{l_ib} Vbar_b + s sum_b e^{l_ib} C_b^T q_i] / sum_b cnt_b e^{l_ib},
+    l_ib = s q_i.Kbar_b (shifted by the row max; the shift cancels)."""
+    out = np.empty((q_rows.shape[0], Vbar_K.shape[1]), dtype=np.float64)
+    cnt = cnt_K.astype(np.float64)
+    for a in range(0, q_rows.shape[0], chunk):
+        qc = q_rows[a:a + chunk]
+        l = scale * (qc @ Kbar_K.T)
+        e = np.exp(l - l.max(axis=1, keepdims=True))
+        num = (e * cnt[None, :]) @ Vbar_K + scale * np.einsum("ib,bde,id->ie", e, C_K, qc)
+        out[a:a + chunk] = num / (e * cnt[None, :]).sum(axis=1, keepdims=True)
+    return out
+
+
+# ---------------------------------------------------------------------------
 # The whole forward for one (b, h)
 # ---------------------------------------------------------------------------
 
 def isa_head(q, k, v, N_src, blk, keep, rho, scale=None,
-             kept_override=None, routed_override=None, rows=None, granularity="token"):
+             kept_override=None, routed_override=None, rows=None, granularity="token",
+             taylor_order=0):
     """ISA forward for one head, all stages in order; float64 inputs [N, d].
 
     ``kept_override`` / ``routed_override`` replace the selected context
@@ -238,6 +278,8 @@ def isa_head(q, k, v, N_src, blk, keep, rho, scale=None,
     ``granularity`` selects the dynamic query grouping: "token" routes the
     n_route sharpest queries one by one; "block" routes whole query blocks
     (see ``route_query_blocks``).
+    ``taylor_order`` 0 (the method) or 1 (``taylor1_rows``) for the rows
+    that are not routed.
     Returns a dict of every intermediate and the output.
     """
     N, d = q.shape
@@ -281,7 +323,14 @@ def isa_head(q, k, v, N_src, blk, keep, rho, scale=None,
     if len(r_sel):
         out[r_sel] = full_rows(q[r_sel], k[T], v[T], s)
     if len(t_sel):
-        out[t_sel] = taylor_rows(q[t_sel], Kbar[Kb], Vbar[Kb], cnts[Kb], s)
+        if taylor_order == 0:
+            out[t_sel] = taylor_rows(q[t_sel], Kbar[Kb], Vbar[Kb], cnts[Kb], s)
+        elif taylor_order == 1:
+            C = correction_matrices(k, v, starts, cnts, Kb)
+            extra["C"] = C
+            out[t_sel] = taylor1_rows(q[t_sel], Kbar[Kb], Vbar[Kb], C, cnts[Kb], s)
+        else:
+            raise ValueError(taylor_order)
     return dict(out=out, Qbar=Qbar, Kbar=Kbar, Vbar=Vbar, cnts=cnts, nSB=nSB, nCB=nCB,
                 sal_all=sal_all, sal_ctx=sal_ctx, kept_ctx=kept_ctx, kept_blocks=Kb,
                 sharp=sharp, routed=routed, taylor=taylor, tokens=T,
