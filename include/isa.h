@@ -180,6 +180,35 @@ int isa_route_blocks_taylor_fwd(const isa_shape* shape, const uint16_t* q, const
 int isa_forward_blocks(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                        uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
+/* First-order Taylor variant of stage 4.  The abstract names its
+ * approximation "0-th order"; the next order keeps the linear term of exp
+ * around the block mean, exp(s q.k_j) ~= exp(s q.Kbar_b)(1 + s q.(k_j -
+ * Kbar_b)) for j in kept block b, which gives
+ *   o_i = [sum_b cnt_b e_ib Vbar_b + s sum_b e_ib C_b^T q_i] / sum_b cnt_b e_ib,
+ *   e_ib = exp(s q_i.Kbar_b),  C_b = sum_{j in b} (k_j - Kbar_b) v_j^T (d x d).
+ * Costs about d/2 times the 0-th order pass (one d x d product per query
+ * and kept block) and is closer to full attention.
+ *
+ * isa_taylor1_workspace_size: bytes of the second workspace `cws` these
+ * calls need: the correction matrices C_b of every kept block, bf16
+ * [B, H, nSB + n_keep, d, d] row-major ([d_in][d_out]); 0 if invalid.
+ *
+ * isa_taylor1_attn_fwd: writes the first-order Taylor output of the
+ * taylor_idx [B, H, N - n_route] rows of out (entries of -1 are padding),
+ * from q, k, v, the kept set and the block means in ws (isa_preselect_ctx
+ * first, same ws).  cws (16-byte aligned, >= isa_taylor1_workspace_size
+ * bytes, else ISA_ERR_WORKSPACE) receives the C_b.
+ *
+ * isa_forward_taylor1: the forward with this variant: isa_preselect_ctx,
+ * isa_route_queries, full attention for the routed rows, first-order
+ * Taylor for the others; index sets held inside ws. */
+size_t isa_taylor1_workspace_size(const isa_shape* shape);
+int isa_taylor1_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const int32_t* kept_ctx_idx, const int32_t* taylor_idx, uint16_t* out,
+                         void* ws, size_t ws_bytes, void* cws, size_t cws_bytes, void* stream);
+int isa_forward_taylor1(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        uint16_t* out, void* ws, size_t ws_bytes, void* cws, size_t cws_bytes, void* stream);
+
 /* All four stages in order on one stream (isa_preselect_ctx,
  * isa_route_taylor_fwd, isa_full_attn_fwd), with the kept set and the
  * routed and Taylor index sets held inside ws.  out [B, H, N, d] bf16. */

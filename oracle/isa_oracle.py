@@ -255,7 +255,9 @@ def taylor1_rows(q_rows, Kbar_K, Vbar_K, C_K, cnt_K, scale, chunk=1024):
         qc = q_rows[a:a + chunk]
         l = scale * (qc @ Kbar_K.T)
         e = np.exp(l - l.max(axis=1, keepdims=True))
-        num = (e * cnt[None, :]) @ Vbar_K + scale * np.einsum("ib,bde,id->ie", e, C_K, qc)
+        num = (e * cnt[None, :]) @ Vbar_K
+        for b in range(len(cnt)):  # s * e_ib * (C_b^T q_i), one kept block at a time
+            num += (scale * e[:, b:b + 1]) * (qc @ C_K[b])
         out[a:a + chunk] = num / (e * cnt[None, :]).sum(axis=1, keepdims=True)
     return out
 

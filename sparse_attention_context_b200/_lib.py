@@ -49,6 +49,9 @@ SIGNATURES = {
     "isa_full_attn_rows_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "isa_route_blocks_taylor_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_forward_blocks": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
+    "isa_taylor1_workspace_size": (_SZ, [_SH]),
+    "isa_taylor1_attn_fwd": (_I, [_SH, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _SZ, _P]),
+    "isa_forward_taylor1": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P, _SZ, _P]),
     "isa_forward": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_forward_static": (_I, [_SH, _P, _P, _P, _P, _P]),
     "isa_dense_workspace_size": (_SZ, [_I]),

@@ -191,6 +191,41 @@ def isa_forward_blocks(q, k, v, N_src: int, block: int, keep: float, rho: float,
     return o
 
 
+def taylor1_workspace(shape: IsaShape, device="cuda") -> torch.Tensor:
+    """Buffer for the correction matrices of the first-order Taylor variant."""
+    n = lib().isa_taylor1_workspace_size(ctypes.byref(shape))
+    if n == 0:
+        raise ValueError("invalid or unsupported shape")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def isa_taylor1_attn_fwd(q, k, v, kept, taylor, shape: IsaShape, ws, cws, out, stream=None):
+    """First-order Taylor output for the taylor rows of `out` (C_b land in cws)."""
+    _check_qkv(q, k, v, out)
+    rc = lib().isa_taylor1_attn_fwd(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                    _ptr(kept) if kept.numel() else None, _ptr(taylor) if taylor.numel() else None,
+                                    out.data_ptr(), ws.data_ptr(), ws.numel(), cws.data_ptr(), cws.numel(),
+                                    _stream(stream))
+    check("isa_taylor1_attn_fwd", rc)
+    return out
+
+
+def isa_forward_taylor1(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, ws=None,
+                        cws=None, out=None, stream=None):
+    """The ISA forward with first-order Taylor attention for the rows that are not routed."""
+    shape = make_shape(q, N_src, block, keep, rho, scale)
+    if ws is None:
+        ws = new_workspace(shape, q.device)
+    if cws is None:
+        cws = taylor1_workspace(shape, q.device)
+    o = torch.empty_like(q) if out is None else out
+    _check_qkv(q, k, v, o)
+    rc = lib().isa_forward_taylor1(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   ws.data_ptr(), ws.numel(), cws.data_ptr(), cws.numel(), _stream(stream))
+    check("isa_forward_taylor1", rc)
+    return o
+
+
 def isa_forward(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, ws=None, out=None,
                 stream=None, groups=None):
     """All ISA stages in one call.

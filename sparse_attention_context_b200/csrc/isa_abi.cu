@@ -326,6 +326,40 @@ int run_taylor(const Ctx& c, const uint16_t* q, const int32_t* kept, const int32
   return cuda_status(e);
 }
 
+// First-order Taylor for the taylor_idx rows: the correction matrices of
+// the kept blocks into cws, then the first-order pass.  The gathered kept
+// operands (Khi, Vb, bias2) must be current (run_build_kept).
+int run_taylor1(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kept,
+                const int32_t* taylor, uint16_t* out, uint16_t* cws) {
+  const Dims& d = c.d;
+  CUtensorMap tmK, tmV;
+  if (!make_tmap_bf16(&tmK, k, static_cast<uint64_t>(d.BH) * d.N, d.d, d.blk) ||
+      !make_tmap_bf16(&tmV, v, static_cast<uint64_t>(d.BH) * d.N, d.d, d.blk))
+    return ISA_ERR_CUDA;
+  cudaError_t e = launch_cbuild(d.d, tmK, tmV, at<float>(c.ws, c.L.Kbar), at<float>(c.ws, c.L.Vbar), kept, cws, d.BH,
+                                d.N_src, d.N_ctx, d.blk, d.n_keep, c.status(), c.st);
+  if (e != cudaSuccess || d.N - d.n_route <= 0) return cuda_status(e);
+  CUtensorMap tmKb, tmVb, tmC;
+  const uint64_t kv_rows = static_cast<uint64_t>(d.BH) * d.nKpad;
+  if (!make_tmap_bf16(&tmKb, at<uint16_t>(c.ws, c.L.Khi), kv_rows, d.d, 128) ||
+      !make_tmap_bf16(&tmVb, at<uint16_t>(c.ws, c.L.Vb), kv_rows, d.d, 128) ||
+      !make_tmap_bf16(&tmC, cws, static_cast<uint64_t>(d.BH) * d.nK * d.d, d.d, d.d))
+    return ISA_ERR_CUDA;
+  FlashParams p = base_params(c);
+  p.q = q;
+  p.out = out;
+  p.row_idx = taylor;
+  p.n_rows = d.N - d.n_route;
+  p.n_kv_tiles = d.nKpad / 128;
+  p.kv_rows_per_head = d.nKpad;
+  p.bias2 = at<float>(c.ws, c.L.bias2);
+  return cuda_status(launch_taylor1(d.d, tmKb, tmVb, tmC, p, d.nK, d.scale, d.BH, c.st));
+}
+
+size_t taylor1_bytes(const Dims& d) {
+  return align256(static_cast<size_t>(d.BH) * d.nK * d.d * d.d * 2);
+}
+
 int run_attn(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kept,
              const int32_t* routed, const int32_t* taylor, uint16_t* out, bool rebuild_kept) {
   int rc = run_full(c, q, k, v, kept, routed, out);
@@ -534,6 +568,48 @@ int isa_forward_blocks(const isa_shape* shape, const uint16_t* q, const uint16_t
   rc = run_preselect(c, q, k, v, kept, nullptr);
   if (rc == ISA_OK) rc = run_route_blocks_taylor(c, q, kept, rblk, rrows, nullptr, nullptr, out);
   if (rc == ISA_OK) rc = run_full_rows(c, q, k, v, kept, rrows, c.d.n_rb * c.d.blk, out);
+  return rc;
+}
+
+size_t isa_taylor1_workspace_size(const isa_shape* shape) {
+  Dims d;
+  if (check_shape(shape, &d) != ISA_OK) return 0;
+  return taylor1_bytes(d);
+}
+
+int isa_taylor1_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const int32_t* kept_ctx_idx, const int32_t* taylor_idx, uint16_t* out, void* ws,
+                         size_t ws_bytes, void* cws, size_t cws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
+  if (c.d.n_keep > 0 && (kept_ctx_idx == nullptr || !aligned16(kept_ctx_idx))) return ISA_ERR_INVALID_ARG;
+  if (c.d.N - c.d.n_route > 0 && (taylor_idx == nullptr || !aligned16(taylor_idx))) return ISA_ERR_INVALID_ARG;
+  rc = check_ws(cws, cws_bytes, taylor1_bytes(c.d));
+  if (rc != ISA_OK) return rc;
+  if (static_cast<long long>(c.d.BH) * c.d.nK * c.d.d >= INT_MAX) return ISA_ERR_UNSUPPORTED;
+  rc = run_build_kept(c, kept_ctx_idx);
+  if (rc != ISA_OK) return rc;
+  return run_taylor1(c, q, k, v, kept_ctx_idx, taylor_idx, out, static_cast<uint16_t*>(cws));
+}
+
+int isa_forward_taylor1(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        uint16_t* out, void* ws, size_t ws_bytes, void* cws, size_t cws_bytes, void* stream) {
+  Ctx c;
+  int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
+  if (rc != ISA_OK) return rc;
+  if (!tensors_ok({q, k, v, out})) return ISA_ERR_INVALID_ARG;
+  rc = check_ws(cws, cws_bytes, taylor1_bytes(c.d));
+  if (rc != ISA_OK) return rc;
+  if (static_cast<long long>(c.d.BH) * c.d.nK * c.d.d >= INT_MAX) return ISA_ERR_UNSUPPORTED;
+  int32_t* kept = at<int32_t>(ws, c.L.kept);
+  int32_t* routed = at<int32_t>(ws, c.L.routed);
+  int32_t* taylor = at<int32_t>(ws, c.L.taylor);
+  rc = run_preselect(c, q, k, v, kept, nullptr);
+  if (rc == ISA_OK) rc = run_route(c, q, kept, routed, taylor, nullptr);  // also gathers the kept operands
+  if (rc == ISA_OK) rc = run_full(c, q, k, v, kept, routed, out);
+  if (rc == ISA_OK) rc = run_taylor1(c, q, k, v, kept, taylor, out, static_cast<uint16_t*>(cws));
   return rc;
 }
 

@@ -88,6 +88,16 @@ cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_
                               int blk, int n_keep, int nKpad, int* status, cudaStream_t st);
 cudaError_t launch_route(const float* sharp, int32_t* routed, int32_t* taylor, int BH, int N, int n_route,
                          int* status, cudaStream_t st);
+// First-order Taylor variant (taylor1.cu).  cbuild: C_b = sum_j (k_j - Kbar_b)
+// v_j^T of every kept block, bf16 [BH, nK, D, D] row-major; tmK / tmV over
+// k / v [BH*N, D] with box rows = blk.  taylor1: the rows of p.row_idx;
+// tmK / tmV over the gathered kept Kbar (bf16 hi) / Vbar [BH*nKpad, D] (box
+// 128 rows), tmC over Cout [BH*nK*D, D] (box D rows); p.bias2 = log2 cnt.
+cudaError_t launch_cbuild(int D, const CUtensorMap& tmK, const CUtensorMap& tmV, const float* Kbar,
+                          const float* Vbar, const int32_t* kept, uint16_t* Cout, int BH, int N_src, int N_ctx,
+                          int blk, int n_keep, int* status, cudaStream_t st);
+cudaError_t launch_taylor1(int D, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmC,
+                           const FlashParams& p, int nK, float scale, int BH, cudaStream_t st);
 // Block-granular grouping (route_blocks.cu): routed_blk [BH, n_rb] ascending
 // block indices, routed_rows [BH, n_rb*blk] rows of those blocks (-1 pads),
 // score_out [BH, nB] block mean sharpness or null.
