@@ -374,6 +374,94 @@ def run_block_grouping(args):
         "steps": K, "warmup": W}), flush=True)
 
 
+def run_taylor1(args):
+    """The first-order Taylor variant of stage 4 on the 480p latent workload
+    beside the 0-th order forward: latency of both forwards (CUDA events),
+    the stage split of the first-order forward, the executed TFLOP/s of its
+    first-order stage against the measured bf16 peak, and the approximation
+    error of each against full attention for every query over the same
+    kept tokens (rho = 1).  One JSON line.  Oracle parity of the variant is
+    checked by tests/test_gpu_taylor1.py."""
+    import torch
+
+    from sparse_attention_context_b200 import api
+
+    cfg = CONFIGS[args.config]
+    if args.heads:
+        cfg = cfg.replace(H=args.heads)
+    if args.rho is not None:
+        cfg = cfg.replace(rho=args.rho)
+    if args.keep is not None:
+        cfg = cfg.replace(keep=args.keep)
+    q, k, v = (to_torch_bf16(b).cuda() for b in make_inputs(cfg, seed=0))
+    stream = torch.cuda.current_stream()
+    shape = api.make_shape(q, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    ws = api.new_workspace(shape)
+    cws = api.taylor1_workspace(shape)
+    out0, out1 = torch.empty_like(q), torch.empty_like(q)
+    W, K = max(args.warmup, 3), max(args.steps, 1)
+
+    def timed(fn):
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
+
+    ms0 = timed(lambda: api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws, out=out0))
+    ms1 = timed(lambda: api.isa_forward_taylor1(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws, cws=cws,
+                                                out=out1))
+    nSB, nCB, n_keep, n_route = counts(cfg)
+    kept = torch.empty((cfg.B, cfg.H, n_keep), dtype=torch.int32, device=q.device)
+    routed = torch.empty((cfg.B, cfg.H, n_route), dtype=torch.int32, device=q.device)
+    taylor = torch.empty((cfg.B, cfg.H, cfg.N - n_route), dtype=torch.int32, device=q.device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    acc = np.zeros(4)
+    for it in range(W + K):
+        ev[0].record(stream)
+        api.isa_preselect_ctx(q, k, v, shape, ws, kept=kept, want_saliency=False)
+        ev[1].record(stream)
+        api.isa_route_taylor_fwd(q, kept, shape, ws, out1, routed=routed, taylor=taylor, want_sharpness=False)
+        ev[2].record(stream)
+        api.isa_full_attn_fwd(q, k, v, kept, routed, shape, ws, out1)
+        ev[3].record(stream)
+        api.isa_taylor1_attn_fwd(q, k, v, kept, taylor, shape, ws, cws, out1)
+        ev[4].record(stream)
+        torch.cuda.synchronize()
+        if it >= W:
+            acc += [ev[j].elapsed_time(ev[j + 1]) for j in range(4)]
+    acc /= K
+    assert api.isa_read_device_status(ws) == 0
+    ref = api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, 1.0)  # every query on full attention
+    torch.cuda.synchronize()
+    ref_abs = ref.float().abs().sum().item()
+
+    def err(o, rows=None):
+        d = (o.float() - ref.float()).abs()
+        return {"mean_rel": round(d.sum().item() / ref_abs, 6), "max_abs": round(d.max().item(), 5)}
+
+    BH, d, nK = cfg.B * cfg.H, cfg.d, nSB + n_keep
+    t1_flops = BH * (cfg.N - n_route) * nK * (4.0 * d + 2.0 * d * d) + BH * nK * 2.0 * d * d * cfg.block
+    pk, pk_kind = peaks()
+    ach = t1_flops / (acc[3] * 1e-3) / 1e12
+    print(json.dumps({
+        "variant": "first-order Taylor stage 4", "config": config_dict(cfg, 1),
+        "taylor0_forward_ms": round(ms0, 4), "taylor1_forward_ms": round(ms1, 4),
+        "taylor1_stage_ms": {"preselect": round(acc[0], 4), "sharpness_taylor0_route": round(acc[1], 4),
+                             "full_attn": round(acc[2], 4), "first_order_taylor": round(acc[3], 4)},
+        "first_order_stage_roofline": {"bound": "tensor", "executed_tflop": round(t1_flops / 1e12, 3),
+                                       "achieved": round(ach, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                       "frac": round(ach / pk["bf16_tflops"], 4),
+                                       "peak_kind": f"{pk_kind} burst bf16"},
+        "error_vs_full_over_kept": {"taylor0": err(out0), "taylor1": err(out1)},
+        "steps": K, "warmup": W}), flush=True)
+
+
 def config_dict(cfg, n):
     return {"workload": f"ISA fwd {cfg.name}-latent: B={cfg.B} H={cfg.H} d={cfg.d} N_src={cfg.N_src} "
                         f"N_ctx={cfg.N_ctx} block={cfg.block} keep={cfg.keep} rho={cfg.rho}",
@@ -398,12 +486,17 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="keep x rho latency grid of the sweep workload")
     ap.add_argument("--grouping", default="token", choices=["token", "block"],
                     help="block: time the block-granular query grouping variant beside the per-token one")
+    ap.add_argument("--taylor-order", type=int, default=0, choices=[0, 1],
+                    help="1: time the first-order Taylor variant of stage 4 beside the 0-th order forward")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args)
         return
     if args.grouping == "block":
         run_block_grouping(args)
+        return
+    if args.taylor_order == 1:
+        run_taylor1(args)
         return
     cfg = CONFIGS[args.config]
     if args.heads:

@@ -200,8 +200,9 @@ int isa_forward_blocks(const isa_shape* shape, const uint16_t* q, const uint16_t
  * bytes, else ISA_ERR_WORKSPACE) receives the C_b.
  *
  * isa_forward_taylor1: the forward with this variant: isa_preselect_ctx,
- * isa_route_queries, full attention for the routed rows, first-order
- * Taylor for the others; index sets held inside ws. */
+ * isa_route_taylor_fwd (its 0-th order rows are overwritten), full
+ * attention for the routed rows, first-order Taylor for the others; index
+ * sets held inside ws. */
 size_t isa_taylor1_workspace_size(const isa_shape* shape);
 int isa_taylor1_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                          const int32_t* kept_ctx_idx, const int32_t* taylor_idx, uint16_t* out,

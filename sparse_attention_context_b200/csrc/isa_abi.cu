@@ -607,7 +607,10 @@ int isa_forward_taylor1(const isa_shape* shape, const uint16_t* q, const uint16_
   int32_t* routed = at<int32_t>(ws, c.L.routed);
   int32_t* taylor = at<int32_t>(ws, c.L.taylor);
   rc = run_preselect(c, q, k, v, kept, nullptr);
-  if (rc == ISA_OK) rc = run_route(c, q, kept, routed, taylor, nullptr);  // also gathers the kept operands
+  // the fused sharpness pass (it also gathers the kept operands) writes
+  // 0-th order rows that the first-order pass then overwrites: cheaper than
+  // the stage-by-stage sharpness kernel
+  if (rc == ISA_OK) rc = run_route_taylor(c, q, kept, routed, taylor, nullptr, out);
   if (rc == ISA_OK) rc = run_full(c, q, k, v, kept, routed, out);
   if (rc == ISA_OK) rc = run_taylor1(c, q, k, v, kept, taylor, out, static_cast<uint16_t*>(cws));
   return rc;

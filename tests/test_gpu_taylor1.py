@@ -28,13 +28,19 @@ CASES = {
 }
 
 
-def run_t1(cfg, q, k, v):
+def run_t1(cfg, q, k, v, fused=True):
+    """The isa_forward_taylor1 sequence stage by stage (fused: the sharpness
+    pass of isa_route_taylor_fwd, as the one-call entry point runs it; else
+    isa_route_queries)."""
     shape = api.make_shape(q, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     ws = api.new_workspace(shape)
     cws = api.taylor1_workspace(shape)
     out = torch.empty_like(q)
     kept, _ = api.isa_preselect_ctx(q, k, v, shape, ws)
-    routed, taylor, sharp = api.isa_route_queries(q, kept, shape, ws)
+    if fused:
+        routed, taylor, sharp = api.isa_route_taylor_fwd(q, kept, shape, ws, out)
+    else:
+        routed, taylor, sharp = api.isa_route_queries(q, kept, shape, ws)
     api.isa_full_attn_fwd(q, k, v, kept, routed, shape, ws, out)
     api.isa_taylor1_attn_fwd(q, k, v, kept, taylor, shape, ws, cws, out)
     status = api.isa_read_device_status(ws)
@@ -78,6 +84,18 @@ def test_taylor1_matches_oracle(cuda_ok, name):
     out = api.isa_forward_taylor1(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), g["out_t"].view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged128", "many_tiles"])
+def test_taylor1_after_stage_by_stage_routing(cuda_ok, name):
+    """isa_taylor1_attn_fwd after isa_route_queries (the stage-by-stage
+    sharpness kernel) against the oracle."""
+    cfg = CASES[name]
+    bits, (q, k, v) = inputs(cfg)
+    g = run_t1(cfg, q, k, v, fused=False)
+    assert g["status"] == 0
+    for h in range(cfg.H):
+        compare_head_t1(cfg, bits, g, h)
 
 
 def test_taylor1_480p_sampled(cuda_ok):
