@@ -467,7 +467,14 @@ def config_dict(cfg, n):
                         f"N_ctx={cfg.N_ctx} block={cfg.block} keep={cfg.keep} rho={cfg.rho}",
             "B": cfg.B, "H": cfg.H, "d": cfg.d, "N_src": cfg.N_src, "N_ctx": cfg.N_ctx, "block": cfg.block,
             "keep": cfg.keep, "rho": cfg.rho, "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
-            "l2": f"inputs ({3 * cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e6:.0f} MB) larger than the 126 MB L2, no flush"}
+            "l2": l2_note(cfg)}
+
+
+def l2_note(cfg):
+    mb = 3 * cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e6
+    if mb > 126:
+        return f"inputs ({mb:.0f} MB) larger than the 126 MB L2, no flush"
+    return f"inputs ({mb:.1f} MB) fit in the 126 MB L2 and stay there between steps (warm, no flush)"
 
 
 def main():
