@@ -79,6 +79,8 @@ def full_traffic(args):
 
     if args.config != FULL_TRAFFIC["config"] or args.heads or args.rho is not None or args.keep is not None:
         return None
+    if getattr(args, "shard", "replicas") == "heads" and int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        return None  # a slice of the heads per rank: not the captured launch
     root = os.path.dirname(os.path.abspath(__file__))
     for rel, digest in FULL_TRAFFIC["sources"].items():
         with open(os.path.join(root, rel), "rb") as f:
@@ -462,11 +464,17 @@ def run_taylor1(args):
         "steps": K, "warmup": W}), flush=True)
 
 
-def config_dict(cfg, n):
+def config_dict(cfg, n, shard="replicas"):
+    if n <= 1:
+        par = "single GPU"
+    elif shard == "heads":
+        par = f"heads sharded x{n}"
+    else:
+        par = f"replicas x{n}"
     return {"workload": f"ISA fwd {cfg.name}-latent: B={cfg.B} H={cfg.H} d={cfg.d} N_src={cfg.N_src} "
                         f"N_ctx={cfg.N_ctx} block={cfg.block} keep={cfg.keep} rho={cfg.rho}",
             "B": cfg.B, "H": cfg.H, "d": cfg.d, "N_src": cfg.N_src, "N_ctx": cfg.N_ctx, "block": cfg.block,
-            "keep": cfg.keep, "rho": cfg.rho, "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
+            "keep": cfg.keep, "rho": cfg.rho, "parallelism": par,
             "l2": l2_note(cfg)}
 
 
@@ -493,6 +501,11 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="keep x rho latency grid of the sweep workload")
     ap.add_argument("--grouping", default="token", choices=["token", "block"],
                     help="block: time the block-granular query grouping variant beside the per-token one")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: one replica of the workload per rank (weak scaling, default) or the heads of one "
+                         "problem split over the ranks (strong scaling)")
+    ap.add_argument("--gather", action="store_true",
+                    help="with --shard heads: also time the all-gather of the output heads onto every rank")
     ap.add_argument("--taylor-order", type=int, default=0, choices=[0, 1],
                     help="1: time the first-order Taylor variant of stage 4 beside the 0-th order forward")
     args = ap.parse_args()
@@ -535,7 +548,19 @@ def main():
         if world > 1:
             dist.barrier()
 
-    bits = make_inputs(cfg, seed=replica_seed(rank))
+    cfg_job = cfg  # the problem the report names
+    if args.shard == "heads":
+        # one problem, its heads split over the ranks: every rank draws its own
+        # heads of the same seeded problem (per-head generator streams)
+        from sparse_attention_context_b200.sharding import shard_heads
+
+        h0, h1 = shard_heads(cfg.H, world, rank)
+        if h1 <= h0:
+            raise SystemExit(f"--shard heads: {cfg.H} heads cannot be split over {world} ranks")
+        bits = make_inputs(cfg, seed=0, heads=range(h0, h1))
+        cfg = cfg.replace(H=h1 - h0)
+    else:
+        bits = make_inputs(cfg, seed=replica_seed(rank))
     q, k, v = (to_torch_bf16(b).to(dev) for b in bits)
     shape = api.make_shape(q, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     ws = api.new_workspace(shape, dev)
@@ -632,6 +657,23 @@ def main():
         e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": 3 * q.numel() * 2,
                "d2h_bytes_per_step": q.numel() * 2}
 
+    gather_ms = None
+    if args.shard == "heads" and args.gather and world > 1:
+        from sparse_attention_context_b200.sharding import gather_heads
+
+        full = gather_heads(out)
+        assert full.shape[1] == cfg_job.H
+        torch.cuda.synchronize()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            gather_heads(out)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        gather_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps, dev)
+        del full
+
     pk, pk_kind = peaks()
     full_ms = float(stage_ms[2])
     ach = wm["full_flops"] / (full_ms * 1e-3) / 1e12
@@ -662,9 +704,9 @@ def main():
     if rank == 0:
         rec = {"metric": METRIC, "value": round(ms_max, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": False,
-               "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-               "config": config_dict(cfg, world),
-               "eff_tflops": round(wm["dense_flops"] / (ms_max * 1e-3) / 1e12, 1),
+               "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None, "dtype": "bf16",
+               "data": "synthetic", "config": config_dict(cfg_job, world, args.shard),
+               "eff_tflops": round(work_model(cfg_job, T_mean)["dense_flops"] / (ms_max * 1e-3) / 1e12, 1),
                "dense_ms": None if dense_ms is None else round(dense_ms, 4),
                "isa_over_dense": None if dense_ms is None else round(ms_max / dense_ms, 4),
                "dense_tflops": None if dense_ms is None else round(wm["dense_flops"] / (dense_ms * 1e-3) / 1e12, 1),
@@ -674,6 +716,8 @@ def main():
                "executed_tflop": round((wm["full_flops"] + wm["fused_flops"]) / 1e12, 4),
                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
+        if gather_ms is not None:
+            rec["gather_ms"] = round(gather_ms, 4)
         print(json.dumps(rec), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -1,10 +1,14 @@
-"""Multi-rank plumbing of bench.py, on CPU with the gloo backend (world size 2).
+"""Multi-rank plumbing of bench.py and of the head sharding, on CPU with the
+gloo backend (world size 2).
 
 The ISA forward shards by (b, h) with no exchange step, so the multi-GPU
-path is one replica of the workload per rank plus the timing reduction.
-These tests cover that host logic without a GPU: the max-over-ranks
-reduction every rank takes part in, the per-rank replica inputs, the
-report's parallelism field, and the reference arm's rank-0-only output."""
+path is one replica of the workload per rank (or one problem's heads split
+over the ranks) plus the timing reduction, and, for callers that want the
+whole output everywhere, one all-gather of the output heads.  These tests
+cover that host logic without a GPU: the max-over-ranks reduction every
+rank takes part in, the per-rank replica inputs, the head partition and
+its gather, the report's parallelism field, and the reference arm's
+rank-0-only output."""
 import json
 import os
 import socket
@@ -60,6 +64,68 @@ def test_two_ranks_reduce_timing_and_run_own_replicas(tmp_path):
         assert d["max"] == pytest.approx(2.5)  # every rank reports the slowest rank's time
         assert d["parallelism"] == "replicas x2"
     assert not np.array_equal(res[0]["q_head"], res[1]["q_head"])  # each replica draws its own inputs
+
+
+def _shard_worker(rank, world, port, out_dir):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    from sparse_attention_context_b200.sharding import gather_heads, shard_heads
+    from workloads import CONFIGS, make_inputs, to_torch_bf16
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        cfg = CONFIGS["tiny"].replace(H=4, N_src=96, N_ctx=64)
+        h0, h1 = shard_heads(cfg.H, world, rank)
+        local = to_torch_bf16(make_inputs(cfg, seed=0, heads=range(h0, h1))[0])
+        full = gather_heads(local)  # stands in for the output slices of the per-rank forwards
+        torch.save(full, os.path.join(out_dir, f"full{rank}.pt"))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_shards_gather_to_the_whole_problem(tmp_path):
+    """Each rank draws only its heads of one seeded problem; the gathered
+    slices equal the whole problem drawn in one process, on every rank."""
+    import torch
+
+    from workloads import CONFIGS, make_inputs, to_torch_bf16
+
+    world = 2
+    mp.start_processes(_shard_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    cfg = CONFIGS["tiny"].replace(H=4, N_src=96, N_ctx=64)
+    whole = to_torch_bf16(make_inputs(cfg, seed=0)[0])
+    for r in range(world):
+        got = torch.load(tmp_path / f"full{r}.pt")
+        assert got.shape == whole.shape
+        assert torch.equal(got.view(torch.int16), whole.view(torch.int16))
+
+
+@pytest.mark.parametrize("H,world", [(24, 1), (24, 2), (24, 8), (40, 8), (7, 3), (3, 4)])
+def test_shard_heads_partition(H, world):
+    from sparse_attention_context_b200.sharding import shard_heads
+
+    ranges = [shard_heads(H, world, r) for r in range(world)]
+    assert ranges[0][0] == 0 and ranges[-1][1] == H
+    assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))  # contiguous, no overlap
+    sizes = [b - a for a, b in ranges]
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_config_names_the_parallelism():
+    import bench
+    from workloads import CONFIGS
+
+    cfg = CONFIGS["480p"]
+    assert bench.config_dict(cfg, 1)["parallelism"] == "single GPU"
+    assert bench.config_dict(cfg, 4)["parallelism"] == "replicas x4"
+    assert bench.config_dict(cfg, 4, "heads")["parallelism"] == "heads sharded x4"
 
 
 def test_max_over_ranks_single_process_is_identity():
