@@ -26,7 +26,9 @@
 //    then for every kept block b the warps write A_b = w_b q (their own q
 //    row, bf16) into one of two 64-column TMEM slots and the issuer adds
 //    O += A_b C_b (UMMA, A from TMEM, C_b staged by TMA in a ring shared by
-//    both tiles).  Every MMA accumulates into one O per tile, so the
+//    both tiles).  The Vbar tile of a key tile travels through the same
+//    ring, as the element before the key tile's C_b, so the ring is as deep
+//    as shared memory allows.  Every MMA accumulates into one O per tile, so the
 //    epilogue is O / l.  The running maximum m is re-based only when it
 //    grows by 2^32 (then O is rescaled in TMEM; every earlier MMA is known
 //    complete once S of the next key tile has landed).
@@ -218,12 +220,13 @@ struct T1Cfg {
   static constexpr int Q_BYTES = 128 * D * 2;    // one 128-row query tile
   static constexpr int KT_BYTES = BN * D * 2;    // one Kbar / Vbar tile
   static constexpr int C_BYTES = D * D * 2;      // one correction matrix
-  static constexpr int R = D == 128 ? 3 : 8;     // correction-matrix ring
+  // ring of Vbar tiles and correction matrices (one slot holds either)
+  static constexpr int SLOT = KT_BYTES > C_BYTES ? KT_BYTES : C_BYTES;
+  static constexpr int R = D == 128 ? 4 : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = 2 * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KT_BYTES;
-  static constexpr int OFF_C = OFF_V + KT_BYTES;
-  static constexpr int OFF_BIAS = OFF_C + R * C_BYTES;  // [2][BN] log2 cnt (ring by key tile parity)
+  static constexpr int OFF_C = OFF_K + KT_BYTES;
+  static constexpr int OFF_BIAS = OFF_C + R * SLOT;  // [2][BN] log2 cnt (ring by key tile parity)
   static constexpr int OFF_BAR = OFF_BIAS + 2 * BN * 4;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -232,8 +235,8 @@ struct T1Cfg {
 
 struct T1Bars {
   uint64_t q_full[2];
-  uint64_t k_full, k_empty, v_full, v_empty;
-  uint64_t c_full[8], c_empty[8];
+  uint64_t k_full, k_empty;
+  uint64_t c_full[8], c_empty[8];  // ring of Vbar tiles and correction matrices
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t a_full[2][2];  // [tile][slot]: A written by the tile's 128 threads
@@ -274,7 +277,6 @@ __global__ void __launch_bounds__(320, 1)
   T1Bars* bars = reinterpret_cast<T1Bars*>(smem + C::OFF_BAR);
   const uint32_t aQ = smem_u32(smem + C::OFF_Q);
   const uint32_t aK = smem_u32(smem + C::OFF_K);
-  const uint32_t aV = smem_u32(smem + C::OFF_V);
   const uint32_t aC = smem_u32(smem + C::OFF_C);
   const float* bias_sm = reinterpret_cast<const float*>(smem + C::OFF_BIAS);
 
@@ -297,8 +299,6 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(&bars->k_full, 1);
     mbar_init(&bars->k_empty, 1);
-    mbar_init(&bars->v_full, 1);
-    mbar_init(&bars->v_empty, 1);
     for (int r = 0; r < R; ++r) {
       mbar_init(&bars->c_full[r], 1);
       mbar_init(&bars->c_empty[r], 1);
@@ -324,9 +324,12 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int gb = 0;
+      int ge = 0;  // ring elements issued: per key tile its Vbar tile, then its C_b
       bool ok = true;
       int k_issued = 0;
+      auto slot_ready = [&](int e) -> bool {  // wait until ring slot e % R is free
+        return e < R || t1w(&bars->c_empty[e % R], ((e / R) - 1) & 1, bars, p);
+      };
       for (int t = 0; ok && t < nT; ++t) {
         if (t > 0 && !(ok = t1w(&bars->k_empty, (t - 1) & 1, bars, p))) break;
         const int kr = bh * p.kv_rows_per_head + t * BN;
@@ -334,29 +337,32 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) tma_load_2d(smem + C::OFF_K + c * (BN * 128), &tmK, &bars->k_full, c * 64, kr);
         bulk_load(smem + C::OFF_BIAS + (t & 1) * BN * 4, p.bias2 + kr, BN * 4, &bars->k_full);
-        if (t > 0 && !(ok = t1w(&bars->v_empty, (t - 1) & 1, bars, p))) break;
-        mbar_arrive_expect_tx(&bars->v_full, C::KT_BYTES);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) tma_load_2d(smem + C::OFF_V + c * (BN * 128), &tmV, &bars->v_full, c * 64, kr);
         k_issued = t + 1;
+        if (!(ok = slot_ready(ge))) break;
+        {
+          const int r = ge % R;
+          mbar_arrive_expect_tx(&bars->c_full[r], C::KT_BYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(smem + C::OFF_C + r * C::SLOT + c * (BN * 128), &tmV, &bars->c_full[r], c * 64, kr);
+          ++ge;
+        }
         const int nb = min(BN, nK - t * BN);
-        for (int b = 0; b < nb; ++b, ++gb) {
-          const int r = gb % R;
-          if (gb >= R && !(ok = t1w(&bars->c_empty[r], ((gb / R) - 1) & 1, bars, p))) break;
+        for (int b = 0; b < nb; ++b) {
+          if (!(ok = slot_ready(ge))) break;
+          const int r = ge % R;
           mbar_arrive_expect_tx(&bars->c_full[r], C::C_BYTES);
           const int crow = (bh * nK + t * BN + b) * D;
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(smem + C::OFF_C + r * C::C_BYTES + c * (D * 128), &tmC, &bars->c_full[r], c * 64, crow);
+            tma_load_2d(smem + C::OFF_C + r * C::SLOT + c * (D * 128), &tmC, &bars->c_full[r], c * 64, crow);
+          ++ge;
         }
       }
       // drain this thread's copies still in flight before the CTA may exit
-      if (k_issued > 0) {
-        mbar_wait_bounded(&bars->k_full, (k_issued - 1) & 1, nullptr, kWaitLimitNs);
-        mbar_wait_bounded(&bars->v_full, (k_issued - 1) & 1, nullptr, kWaitLimitNs);
-      }
-      for (int g = gb > R ? gb - R : 0; g < gb; ++g)
-        mbar_wait_bounded(&bars->c_full[g % R], (g / R) & 1, nullptr, kWaitLimitNs);
+      if (k_issued > 0) mbar_wait_bounded(&bars->k_full, (k_issued - 1) & 1, nullptr, kWaitLimitNs);
+      for (int e = ge > R ? ge - R : 0; e < ge; ++e)
+        mbar_wait_bounded(&bars->c_full[e % R], (e / R) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ UMMA issuer
@@ -364,7 +370,7 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t IDS = idesc_bf16(128, BN, 0);
       constexpr uint32_t IDO = idesc_bf16(128, D, 1);
       bool ok = t1w(&bars->q_full[0], 0, bars, p) && t1w(&bars->q_full[1], 0, bars, p);
-      int gb = 0;
+      int ge = 0;  // ring elements consumed (same order as the producer)
       int na[2][2] = {{0, 0}, {0, 0}};
       for (int t = 0; ok && t < nT; ++t) {
         if (!(ok = t1w(&bars->k_full, t & 1, bars, p))) break;
@@ -377,7 +383,9 @@ __global__ void __launch_bounds__(320, 1)
           umma_commit(&bars->s_full[i]);
         }
         umma_commit(&bars->k_empty);
-        if (!(ok = t1w(&bars->v_full, t & 1, bars, p))) break;
+        const int rv = ge % R;
+        if (!(ok = t1w(&bars->c_full[rv], (ge / R) & 1, bars, p))) break;
+        const uint32_t aV = aC + rv * C::SLOT;
         for (int i = 0; i < 2 && ok; ++i) {
           if (!(ok = t1w(&bars->p_full[i], t & 1, bars, p))) break;
           tc_fence_after();
@@ -388,12 +396,13 @@ __global__ void __launch_bounds__(320, 1)
           umma_commit(&bars->a_free[i][0]);
         }
         if (!ok) break;
-        umma_commit(&bars->v_empty);
+        umma_commit(&bars->c_empty[rv]);
+        ++ge;
         const int nb = min(BN, nK - t * BN);
-        for (int b = 0; ok && b < nb; ++b, ++gb) {
-          const int r = gb % R, s = b & 1;
-          if (!(ok = t1w(&bars->c_full[r], (gb / R) & 1, bars, p))) break;
-          const uint32_t cb = aC + r * C::C_BYTES;
+        for (int b = 0; ok && b < nb; ++b, ++ge) {
+          const int r = ge % R, s = b & 1;
+          if (!(ok = t1w(&bars->c_full[r], (ge / R) & 1, bars, p))) break;
+          const uint32_t cb = aC + r * C::SLOT;
           for (int i = 0; i < 2; ++i) {
             if (!(ok = t1w(&bars->a_full[i][s], na[i][s] & 1, bars, p))) break;
             ++na[i][s];
