@@ -464,6 +464,64 @@ def run_taylor1(args):
         "steps": K, "warmup": W}), flush=True)
 
 
+def run_dit_layer(args):
+    """A DiT self-attention layer (QKV projection, attention, output
+    projection; random bf16 weights, C = H*d channels) on the 480p latent
+    shape, with the ISA forward and with the in-house dense kernel as its
+    attention: layer latency and its parts (CUDA events).  One JSON line."""
+    import torch
+
+    from sparse_attention_context_b200 import api
+    from sparse_attention_context_b200.dit_layer import attention_layer, merge_heads, random_weights, split_heads
+
+    cfg = CONFIGS[args.config]
+    if args.heads:
+        cfg = cfg.replace(H=args.heads)
+    H, N, d = cfg.H, cfg.N, cfg.d
+    C = H * d
+    g = torch.Generator(device="cpu").manual_seed(0)
+    x = torch.randn(N, C, generator=g).to(device="cuda", dtype=torch.bfloat16)
+    w_qkv, w_o = random_weights(C)
+    stream = torch.cuda.current_stream()
+    shape = api.make_shape(torch.empty((1, H, N, d), device="meta"), cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    ws = api.new_workspace(shape)
+    dws = api.dense_workspace(d)
+    W, K = max(args.warmup, 3), max(args.steps, 1)
+
+    def timed(fn, k=K):
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / k
+
+    kw = dict(H=H, N_src=cfg.N_src, block=cfg.block, keep=cfg.keep, rho=cfg.rho)
+    isa_ms = timed(lambda: attention_layer(x, w_qkv, w_o, attention="isa", ws=ws, **kw))
+    dense_ms = timed(lambda: attention_layer(x, w_qkv, w_o, attention="dense", dense_ws=dws, **kw), max(2, K // 4))
+    qkv_ms = timed(lambda: split_heads(x @ w_qkv.t(), H))
+    q, k, v = split_heads(x @ w_qkv.t(), H)
+    attn_ms = timed(lambda: api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws))
+    o = api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws)
+    out_ms = timed(lambda: merge_heads(o) @ w_o.t())
+    dense_attn_ms = timed(lambda: api.isa_dense_attn_fwd(q, k, v, ws=dws), max(2, K // 4))
+    assert api.isa_read_device_status(ws) == 0
+    proj_flop = 2.0 * N * C * 3 * C + 2.0 * N * C * C
+    print(json.dumps({
+        "variant": "DiT self-attention layer", "config": config_dict(cfg, 1),
+        "channels": C, "weights": "random bf16 (std 1/sqrt(C))", "input": "x ~ N(0, 1) bf16, seed 0",
+        "layer_isa_ms": round(isa_ms, 4), "layer_dense_ms": round(dense_ms, 4),
+        "layer_isa_over_dense": round(isa_ms / dense_ms, 4),
+        "attention_isa_ms": round(attn_ms, 4), "attention_dense_ms": round(dense_attn_ms, 4),
+        "qkv_projection_ms": round(qkv_ms, 4), "out_projection_ms": round(out_ms, 4),
+        "projection_tflops": round(proj_flop / ((qkv_ms + out_ms) * 1e-3) / 1e12, 1),
+        "steps": K, "warmup": W}), flush=True)
+
+
 def config_dict(cfg, n, shard="replicas"):
     if n <= 1:
         par = "single GPU"
@@ -506,6 +564,8 @@ def main():
                          "problem split over the ranks (strong scaling)")
     ap.add_argument("--gather", action="store_true",
                     help="with --shard heads: also time the all-gather of the output heads onto every rank")
+    ap.add_argument("--dit-layer", action="store_true",
+                    help="time a DiT self-attention layer (projections + ISA) beside the same layer with dense attention")
     ap.add_argument("--taylor-order", type=int, default=0, choices=[0, 1],
                     help="1: time the first-order Taylor variant of stage 4 beside the 0-th order forward")
     args = ap.parse_args()
@@ -517,6 +577,9 @@ def main():
         return
     if args.taylor_order == 1:
         run_taylor1(args)
+        return
+    if args.dit_layer:
+        run_dit_layer(args)
         return
     cfg = CONFIGS[args.config]
     if args.heads:
