@@ -298,39 +298,37 @@ __global__ void __launch_bounds__(320, 1)
         if (!(ok = fwarp(&bars->s_full[i], g & 1, bars, p))) break;
         tc_fence_after();
         const float* bias = reinterpret_cast<const float*>(smem + C::OFF_BIAS + (g & 1) * BN * 4);
-        // logits of half h (64 columns), in log2 units: s*log2(e)*S + log2 cnt
-        auto load_half = [&](int h, float (&x)[64]) {
+        // every S column of the tile in flight at once; the raw scores stay
+        // in registers for both passes.  Logits in log2 units:
+        // x = s*log2(e)*S + log2 cnt (key bias, -inf on padding).
+        uint32_t sreg[BN / 32][32];
 #pragma unroll
-          for (int q2 = 0; q2 < 2; ++q2) {
-            uint32_t u[32];
-            tmem_ld32(sS + h * 64 + q2 * 32, u);
-            tmem_wait_ld();
-            fregs_after(u);
-            const float4* bp = reinterpret_cast<const float4*>(bias + h * 64 + q2 * 32);
+        for (int j = 0; j < BN / 32; ++j) tmem_ld32(sS + j * 32, sreg[j]);
+        tmem_wait_ld();
 #pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4) {
-              const float4 b = bp[c4];
-              const int c = 4 * c4;
-              x[q2 * 32 + c + 0] = fmaf(__uint_as_float(u[c + 0]), p.scale_log2, b.x);
-              x[q2 * 32 + c + 1] = fmaf(__uint_as_float(u[c + 1]), p.scale_log2, b.y);
-              x[q2 * 32 + c + 2] = fmaf(__uint_as_float(u[c + 2]), p.scale_log2, b.z);
-              x[q2 * 32 + c + 3] = fmaf(__uint_as_float(u[c + 3]), p.scale_log2, b.w);
-            }
+        for (int j = 0; j < BN / 32; ++j) fregs_after(sreg[j]);
+        const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+        float pm[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) pm[c] = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) {
+          const float4* bp = reinterpret_cast<const float4*>(bias + j * 32);
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 b = bp[c4];
+            const float2 x01 = __ffma2_rn(
+                make_float2(__uint_as_float(sreg[j][4 * c4]), __uint_as_float(sreg[j][4 * c4 + 1])), sl2,
+                make_float2(b.x, b.y));
+            const float2 x23 = __ffma2_rn(
+                make_float2(__uint_as_float(sreg[j][4 * c4 + 2]), __uint_as_float(sreg[j][4 * c4 + 3])), sl2,
+                make_float2(b.z, b.w));
+            pm[c4] = fmax3(pm[c4], x01.x, x01.y);
+            pm[c4] = fmax3(pm[c4], x23.x, x23.y);
           }
-        };
-        float mt = -INFINITY;
-#pragma unroll
-        for (int h = 0; h < BN / 64; ++h) {
-          float x[64];
-          load_half(h, x);
-          float pm[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) pm[c] = x[c];
-#pragma unroll
-          for (int c = 8; c < 64; ++c) pm[c & 7] = fmaxf(pm[c & 7], x[c]);
-          mt = fmaxf(mt, fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))));
         }
+        const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         mx = fmaxf(mx, mt);
         const float m_new = fmaxf(m, mt);
         // rescale only when the running maximum grew by more than 2^32 (every
@@ -342,24 +340,29 @@ __global__ void __launch_bounds__(320, 1)
           m = m_new;
         }
         const float mref = (m == -INFINITY) ? 0.f : m;
-        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float2 nm2 = make_float2(-mref, -mref);
+        float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int h = 0; h < BN / 64; ++h) {
-          float x[64];
-          load_half(h, x);  // S columns [64h, 64h+64); P of half h goes to columns [32h, 32h+32)
+        for (int j = 0; j < BN / 32; ++j) {
+          // quarter j: P to columns [16j, 16j + 16) (their scores are in registers)
+          const float2* bp = reinterpret_cast<const float2*>(bias + j * 32);
+          uint32_t w[16];
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            uint32_t w[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float e0 = ex2(x[j * 32 + 2 * c] - mref);
-              const float e1 = ex2(x[j * 32 + 2 * c + 1] - mref);
-              ps[(2 * c) & 7] += e0;
-              ps[(2 * c + 1) & 7] += e1;
-              w[c] = pack_bf16(e0, e1);
-            }
-            tmem_st16(sS + h * 32 + j * 16, w);
+          for (int c = 0; c < 16; ++c) {
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(sreg[j][2 * c]), __uint_as_float(sreg[j][2 * c + 1])), sl2, bp[c]);
+            const float2 a = __fadd2_rn(x, nm2);
+            const float e0 = ex2(a.x), e1 = ex2(a.y);
+            ps2[c & 3] = __fadd2_rn(ps2[c & 3], make_float2(e0, e1));
+            w[c] = pack_bf16(e0, e1);
           }
+          tmem_st16(sS + j * 16, w);
+        }
+        float ps[8];
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          ps[2 * k2] = ps2[k2].x;
+          ps[2 * k2 + 1] = ps2[k2].y;
         }
         l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         // O_i rescale (PV_i(g-1) is complete, PV_i(g) not yet issued)
