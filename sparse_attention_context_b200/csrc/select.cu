@@ -11,9 +11,12 @@
 //
 // saliency_kernel: grid (ceil(nB/32), B*H); a CTA owns 32 query blocks and
 //   walks the key blocks in tiles of 64 staged in shared memory (each K-bar
-//   row is read from L2 once per pass per CTA), computing the logits in fp32
-//   (two passes: row max and sum, then the column contributions; logits
-//   recomputed bit-identically), and writes per-chunk partial column sums.
+//   row is read from L2 once per CTA), computing the logits in fp32 (pass 1:
+//   row max and sum; pass 2: the column contributions of the context
+//   blocks), and writes per-chunk partial column sums.  Pass 1 keeps its
+//   logits in shared memory when 32 x nB floats fit, so pass 2 reads them
+//   back instead of recomputing them; larger shapes recompute them
+//   bit-identically.
 // select_ctx_kernel: one 1024-thread CTA per (b, h); sums the partials in a
 //   fixed order, bitonic-sorts (saliency, block) keys in shared memory, and
 //   writes the kept block numbers in ascending order.
@@ -39,8 +42,13 @@ template <int D>
 constexpr int sal_smem_bytes() {
   return (kSalRows * D + kSalColTile * (D + 4) + 16 * kSalColTile) * 4;
 }
+// Shared memory of the logit cache: kSalRows rows of nB logits, padded to
+// whole column tiles.
+inline size_t sal_cache_bytes(int nB) {
+  return static_cast<size_t>(kSalRows) * ((nB + kSalColTile - 1) / kSalColTile * kSalColTile) * 4;
+}
 
-template <int D>
+template <int D, bool CACHE>
 __global__ void __launch_bounds__(256) saliency_kernel(const float* __restrict__ Qbar, const float* __restrict__ Kbar,
                                                        float* __restrict__ partial, int N_src, int N_ctx, int blk,
                                                        int nSB, int nB, float scale) {
@@ -51,6 +59,8 @@ __global__ void __launch_bounds__(256) saliency_kernel(const float* __restrict__
   float* sQ = sal_sm;               // [RB][D]
   float* sK = sQ + RB * D;          // [CT][KP]
   float* sRed = sK + CT * KP;       // [16][CT] column partial sums of the 16 row pairs
+  float* sL = sRed + 16 * CT;       // CACHE: [RB][nBp] logits of pass 1
+  const int nBp = (nB + CT - 1) / CT * CT;
   const int chunk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int ty = tid >> 4, tx = tid & 15;  // rows 2ty, 2ty+1; tile columns tx + 16m
   const int nCB = nB - nSB;
@@ -116,6 +126,12 @@ __global__ void __launch_bounds__(256) saliency_kernel(const float* __restrict__
     __syncthreads();
     float lg[2][4];
     tile_logits(c0, lg);
+    if constexpr (CACHE) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) sL[(2 * ty + i) * nBp + c0 + tx + 16 * m] = lg[i][m];
+    }
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -149,11 +165,25 @@ __global__ void __launch_bounds__(256) saliency_kernel(const float* __restrict__
   // Pass 2: column contributions sum_r cnt_r * P_rc for the context blocks
   float* out = partial + (static_cast<size_t>(bh) * gridDim.x + chunk) * nCB;
   for (int c0 = nSB; c0 < nB; c0 += CT) {
-    __syncthreads();
-    stage(c0);
-    __syncthreads();
     float lg[2][4];
-    tile_logits(c0, lg);
+    if constexpr (CACHE) {
+      // the logits of pass 1: the same rows, columns possibly written by
+      // another thread of the row pair (pass 2 tiles start at nSB); the
+      // barrier makes them visible and also guards sRed of the previous tile
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int c = c0 + tx + 16 * m;
+          lg[i][m] = c < nB ? sL[(2 * ty + i) * nBp + c] : -INFINITY;
+        }
+    } else {
+      __syncthreads();
+      stage(c0);
+      __syncthreads();
+      tile_logits(c0, lg);
+    }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       float col = 0.f;
@@ -274,18 +304,21 @@ cudaError_t launch_saliency(const float* Qbar, const float* Kbar, float* partial
   if (nCB == 0) return cudaSuccess;
   const dim3 grid((nB + kSalRows - 1) / kSalRows, BH);
   cudaError_t e;
+  auto run = [&](auto kern, size_t smem) -> cudaError_t {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    kern<<<grid, 256, smem, st>>>(Qbar, Kbar, partial, N_src, N_ctx, blk, nSB, nB, scale);
+    return cudaGetLastError();
+  };
+  constexpr size_t kMax = 227 * 1024;
   if (D == 128) {
-    constexpr int smem = sal_smem_bytes<128>();
-    if ((e = cudaFuncSetAttribute(saliency_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-      return e;
-    saliency_kernel<128><<<grid, 256, smem, st>>>(Qbar, Kbar, partial, N_src, N_ctx, blk, nSB, nB, scale);
+    const size_t base = sal_smem_bytes<128>(), cached = base + sal_cache_bytes(nB);
+    e = cached <= kMax ? run(saliency_kernel<128, true>, cached) : run(saliency_kernel<128, false>, base);
   } else {
-    constexpr int smem = sal_smem_bytes<64>();
-    if ((e = cudaFuncSetAttribute(saliency_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-      return e;
-    saliency_kernel<64><<<grid, 256, smem, st>>>(Qbar, Kbar, partial, N_src, N_ctx, blk, nSB, nB, scale);
+    const size_t base = sal_smem_bytes<64>(), cached = base + sal_cache_bytes(nB);
+    e = cached <= kMax ? run(saliency_kernel<64, true>, cached) : run(saliency_kernel<64, false>, base);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_select_ctx(const float* partial, float* sal_ws, float* sal_user, int32_t* kept, int BH,
