@@ -26,6 +26,7 @@ CASES = {
     "no_context": CONFIGS["tiny"].replace(N_ctx=0, N_src=300),
     "src_lt_block": CONFIGS["tiny"].replace(N_src=30, N_ctx=400, block=128, keep=0.5, rho=0.5),
     "many_tiles": CONFIGS["tiny"].replace(H=1, d=128, N_src=3000, N_ctx=2900, block=128, keep=0.35, rho=0.25),
+    "batch2": CONFIGS["tiny"].replace(B=2, H=3, d=128, N_src=700, N_ctx=450, block=128, keep=0.5, rho=0.2),
 }
 
 
@@ -49,25 +50,25 @@ def expected_rows(blocks, starts, cnts, blk):
     return rows
 
 
-def compare_head_blocks(cfg, bits, g, h, rows=None):
-    q, k, v = (bf16_bits_to_f64(x[0, h]) for x in bits)
+def compare_head_blocks(cfg, bits, g, b, h, rows=None):
+    q, k, v = (bf16_bits_to_f64(x[b, h]) for x in bits)
     ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, granularity="block", rows=rows)
     nk, nrb = ref["n_keep"], ref["n_route_blocks"]
-    kept = g["kept"][0, h] if nk else np.zeros(0, np.int64)
+    kept = g["kept"][b, h] if nk else np.zeros(0, np.int64)
     if not check_set(kept, ref["kept_ctx"], ref["sal_ctx"], nk):
         ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, granularity="block",
                               kept_override=kept, rows=rows)
-    assert np.allclose(g["sharp"][0, h], ref["sharp"], rtol=1e-4, atol=1e-7), "sharpness"
-    assert np.allclose(g["score"][0, h], ref["block_score"], rtol=1e-4, atol=1e-7), "block scores"
-    rblk = g["rblk"][0, h] if nrb else np.zeros(0, np.int64)
+    assert np.allclose(g["sharp"][b, h], ref["sharp"], rtol=1e-4, atol=1e-7), "sharpness"
+    assert np.allclose(g["score"][b, h], ref["block_score"], rtol=1e-4, atol=1e-7), "block scores"
+    rblk = g["rblk"][b, h] if nrb else np.zeros(0, np.int64)
     assert np.all(np.diff(rblk) > 0), "routed blocks not ascending"
     if not check_set(rblk, ref["routed_blocks"], ref["block_score"], nrb):
         ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, granularity="block",
                               kept_override=kept, routed_override=rblk, rows=rows)
     starts, cnts = oracle.block_layout(cfg.N_src, cfg.N_ctx, cfg.block)[:2]
-    assert g["rows"][0, h].tolist() == expected_rows(rblk, starts, cnts, cfg.block).tolist(), "row list"
+    assert g["rows"][b, h].tolist() == expected_rows(rblk, starts, cnts, cfg.block).tolist(), "row list"
     sel = slice(None) if rows is None else rows
-    return check_out(g["out"][0, h][sel], ref["out"][sel], f"out h{h}")
+    return check_out(g["out"][b, h][sel], ref["out"][sel], f"out b{b} h{h}")
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -76,8 +77,9 @@ def test_block_grouping_matches_oracle(cuda_ok, name):
     bits, (q, k, v) = inputs(cfg)
     g = run_blocks(cfg, q, k, v)
     assert g["status"] == 0
-    for h in range(cfg.H):
-        compare_head_blocks(cfg, bits, g, h)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            compare_head_blocks(cfg, bits, g, b, h)
     # the one-call entry point runs the same kernels: identical bits
     out = api.isa_forward_blocks(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     torch.cuda.synchronize()
@@ -95,7 +97,7 @@ def test_block_grouping_480p_sampled(cuda_ok):
     for h in (0, cfg.H - 1):
         rows = np.unique(np.concatenate([rng.choice(cfg.N, 192, replace=False),
                                          [0, cfg.N_src - 1, cfg.N_src, cfg.N - 1]]))
-        compare_head_blocks(cfg, bits, g, h, rows=rows)
+        compare_head_blocks(cfg, bits, g, 0, h, rows=rows)
 
 
 def test_padding_rows_are_never_stored(cuda_ok):

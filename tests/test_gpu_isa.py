@@ -27,6 +27,7 @@ CASES = {
     "ctx_lt_block": CONFIGS["tiny"].replace(N_src=200, N_ctx=50, keep=1.0),
     "src_lt_block": CONFIGS["tiny"].replace(N_src=30, N_ctx=400, block=128, keep=0.5),
     "many_tiles": CONFIGS["tiny"].replace(H=1, d=128, N_src=3000, N_ctx=2900, block=128, keep=0.35, rho=0.25),
+    "batch2": CONFIGS["tiny"].replace(B=2, H=3, d=128, N_src=700, N_ctx=450, block=128, keep=0.5, rho=0.2),
 }
 
 

@@ -25,6 +25,7 @@ CASES = {
     "no_ctx_kept": CONFIGS["tiny"].replace(keep=0.0),
     "many_tiles": CONFIGS["tiny"].replace(H=1, d=128, N_src=3000, N_ctx=2900, block=128, keep=0.35, rho=0.25),
     "two_key_tiles": CONFIGS["tiny"].replace(H=1, d=64, N_src=9000, N_ctx=9000, block=64, keep=0.5, rho=0.2),
+    "batch2": CONFIGS["tiny"].replace(B=2, H=3, d=128, N_src=700, N_ctx=450, block=128, keep=0.5, rho=0.2),
 }
 
 
@@ -51,25 +52,25 @@ def run_t1(cfg, q, k, v, fused=True):
                 out=bf16_bits_to_f64(from_torch_bf16(out)), status=status)
 
 
-def compare_head_t1(cfg, bits, g, h, rows=None):
-    q, k, v = (bf16_bits_to_f64(x[0, h]) for x in bits)
+def compare_head_t1(cfg, bits, g, b, h, rows=None):
+    q, k, v = (bf16_bits_to_f64(x[b, h]) for x in bits)
     kw = dict(taylor_order=1, rows=rows)
     ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, **kw)
     nk, nr = ref["n_keep"], ref["n_route"]
-    kept = g["kept"][0, h] if nk else np.zeros(0, np.int64)
+    kept = g["kept"][b, h] if nk else np.zeros(0, np.int64)
     if not check_set(kept, ref["kept_ctx"], ref["sal_ctx"], nk):
         ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, kept_override=kept, **kw)
-    routed = g["routed"][0, h] if nr else np.zeros(0, np.int64)
+    routed = g["routed"][b, h] if nr else np.zeros(0, np.int64)
     if not check_set(routed, ref["routed"], ref["sharp"], nr):
         ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, kept_override=kept,
                               routed_override=routed, **kw)
     if "C" in ref:
-        Cg, Cr = g["C"][h], ref["C"]
+        Cg, Cr = g["C"][b * cfg.H + h], ref["C"]
         # bf16 storage of each entry: relative 2^-9, plus fp32 accumulation
         assert np.allclose(Cg, Cr, rtol=5e-3, atol=1e-3 * np.abs(Cr).max()), \
             f"C max err {np.abs(Cg - Cr).max():.3e} of max {np.abs(Cr).max():.2f}"
     sel = slice(None) if rows is None else rows
-    return check_out(g["out"][0, h][sel], ref["out"][sel], f"taylor1 out h{h}")
+    return check_out(g["out"][b, h][sel], ref["out"][sel], f"taylor1 out b{b} h{h}")
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -78,8 +79,9 @@ def test_taylor1_matches_oracle(cuda_ok, name):
     bits, (q, k, v) = inputs(cfg)
     g = run_t1(cfg, q, k, v)
     assert g["status"] == 0
-    for h in range(cfg.H):
-        compare_head_t1(cfg, bits, g, h)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            compare_head_t1(cfg, bits, g, b, h)
     # the one-call entry point runs the same kernels: identical bits
     out = api.isa_forward_taylor1(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     torch.cuda.synchronize()
@@ -94,8 +96,9 @@ def test_taylor1_after_stage_by_stage_routing(cuda_ok, name):
     bits, (q, k, v) = inputs(cfg)
     g = run_t1(cfg, q, k, v, fused=False)
     assert g["status"] == 0
-    for h in range(cfg.H):
-        compare_head_t1(cfg, bits, g, h)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            compare_head_t1(cfg, bits, g, b, h)
 
 
 def test_taylor1_480p_sampled(cuda_ok):
@@ -109,7 +112,7 @@ def test_taylor1_480p_sampled(cuda_ok):
     for h in (0, cfg.H - 1):
         rows = np.unique(np.concatenate([rng.choice(cfg.N, 160, replace=False),
                                          [0, cfg.N_src - 1, cfg.N_src, cfg.N - 1]]))
-        compare_head_t1(cfg, bits, g, h, rows=rows)
+        compare_head_t1(cfg, bits, g, 0, h, rows=rows)
 
 
 def test_taylor1_injected_timeout_is_reported(cuda_ok):
