@@ -18,10 +18,23 @@
 //     counts of equal-to-T and of routed keys are scanned CTA-wide in (j,
 //     warp) order, so every key gets its rank among equal keys and then its
 //     output slot from a warp ballot; both buckets are written coalesced.
+//
+// route_cluster_kernel (used whenever a head's keys fit): the same select
+// and compaction spread over a cluster of 8 CTAs per (b, h), each holding a
+// contiguous eighth of the head's keys in shared memory.  Every radix pass
+// builds the chunk's histogram, the cluster synchronises, and every CTA
+// sums the 8 histograms over distributed shared memory and takes the same
+// (deterministic) decision; the compaction offsets of a chunk come from
+// the greater-than and equal-to-T counts of the chunks before it.  The
+// index sets are identical to the single-CTA kernel's.
+#include <cooperative_groups.h>
+
 #include "block_scan.cuh"
 #include "isa_internal.h"
 
 namespace isa {
+
+namespace cg = cooperative_groups;
 
 // Dynamic shared memory: the resident keys (N words, when they fit) and two
 // count arrays of ceil(N/1024)*32 ints; the static part (histograms, scan
@@ -180,12 +193,257 @@ __global__ void __launch_bounds__(1024) route_kernel(const float* __restrict__ s
   }
 }
 
+constexpr int kRouteCluster = 8;    // CTAs per (b, h)
+constexpr int kRouteCT = 512;       // threads per CTA
+constexpr int kRouteNW = kRouteCT / 32;
+constexpr int kRouteChunkCap = (200 * 1024) / 4 - 2048;  // keys per CTA held in shared memory
+
+// Exclusive prefix sum of v over the kRouteCT threads in thread order;
+// `total` receives the CTA-wide sum.  ws: >= 32 ints of shared memory.
+__device__ __forceinline__ int block_exclusive_sum_512(int v, int* ws, int& total) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) ws[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int t = lane < kRouteNW ? ws[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += n;
+    }
+    if (lane < kRouteNW) ws[lane] = t;  // inclusive over warps
+  }
+  __syncthreads();
+  const int off = w ? ws[w - 1] : 0;
+  total = ws[kRouteNW - 1];
+  __syncthreads();  // ws may be reused right after
+  return off + incl - v;
+}
+
+__global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT)
+    route_cluster_kernel(const float* __restrict__ sharp, int32_t* __restrict__ routed, int32_t* __restrict__ taylor,
+                         int N, int n_route, int* __restrict__ status) {
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = static_cast<int>(cl.block_rank());
+  const int bh = static_cast<int>(blockIdx.x) / kRouteCluster;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int chunk = (N + kRouteCluster - 1) / kRouteCluster;
+  const int c0 = min(N, rank * chunk);
+  const int n = max(0, min(N, c0 + chunk) - c0);  // keys of this CTA: [c0, c0 + n)
+  const int trips = (chunk + kRouteCT - 1) / kRouteCT;
+  extern __shared__ unsigned rkeys[];                        // [chunk]
+  int* ceq = reinterpret_cast<int*>(rkeys + chunk);          // [trips][NW] equal-to-T keys, then offsets
+  int* csel = ceq + trips * kRouteNW;                        // [trips][NW] routed keys, then offsets
+  __shared__ int whist[kRouteNW][257];                       // per warp, padded
+  __shared__ int hist[2][256];                               // this chunk's histogram, by pass parity
+  __shared__ int cnt2[2];                                    // keys > T, keys == T of this chunk
+  __shared__ unsigned sh_sel;
+  __shared__ int sh_rem;
+  __shared__ int sh_off[2];                                  // routed keys before this chunk, equal keys it takes
+  __shared__ int scan_ws[32];
+  const unsigned* u = reinterpret_cast<const unsigned*>(sharp + static_cast<size_t>(bh) * N);
+  for (int i = tid; i < n; i += kRouteCT) rkeys[i] = __ldg(u + c0 + i);
+  __syncthreads();
+
+  unsigned T = 0u;
+  int need_eq = 0;
+  const bool partial = n_route > 0 && n_route < N;  // uniform over the cluster
+  if (partial) {
+    unsigned prefix = 0u, pmask = 0u;
+    int remaining = n_route;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass, buf = pass & 1;
+      for (int e = tid; e < kRouteNW * 257; e += kRouteCT) (&whist[0][0])[e] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += kRouteCT) {
+        const unsigned x = rkeys[i];
+        if ((x & pmask) == prefix) atomicAdd(&whist[w][(x >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (tid < 256) {
+        int t = 0;
+#pragma unroll
+        for (int ww = 0; ww < kRouteNW; ++ww) t += whist[ww][tid];
+        hist[buf][tid] = t;
+      }
+      // every chunk's histogram of this pass is complete (and every read of
+      // the other buffer, two passes back, is done)
+      cl.sync();
+      if (w == 0) {
+        // lane l owns bins 255-8l .. 248-8l (descending): the cluster-wide
+        // counts, then the bin where the count from the top reaches `remaining`
+        int tot[8];
+        int s = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int bin = 255 - 8 * lane - k;
+          int t = 0;
+#pragma unroll
+          for (int r = 0; r < kRouteCluster; ++r) t += cl.map_shared_rank(&hist[buf][0], r)[bin];
+          tot[k] = t;
+          s += t;
+        }
+        int incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int nn = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += nn;
+        }
+        const int before = incl - s;
+        if (before < remaining && incl >= remaining) {  // exactly one lane
+          int cum = before;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if (cum + tot[k] >= remaining) {
+              sh_sel = static_cast<unsigned>(255 - 8 * lane - k);
+              sh_rem = remaining - cum;
+              break;
+            }
+            cum += tot[k];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= sh_sel << shift;
+      pmask |= 255u << shift;
+      remaining = sh_rem;
+      __syncthreads();
+    }
+    T = prefix;
+    need_eq = remaining;
+  }
+
+  // per (trip, warp): keys equal to T (for their rank among equal keys) and
+  // keys above T; the chunk's totals go to the cluster
+  int gt = 0;
+  for (int j = 0; j < trips; ++j) {
+    const int i = j * kRouteCT + tid;
+    const unsigned x = i < n ? rkeys[i] : 0u;
+    const unsigned beq = __ballot_sync(0xffffffffu, partial && i < n && x == T);
+    const unsigned bgt = __ballot_sync(0xffffffffu, partial && i < n && x > T);
+    if (lane == 0) {
+      ceq[j * kRouteNW + w] = __popc(beq);
+      gt += __popc(bgt);
+    }
+  }
+  __syncthreads();
+  {
+    const int per = (trips * kRouteNW + kRouteCT - 1) / kRouteCT;
+    int loc = 0;
+    for (int k = 0; k < per; ++k) {
+      const int e = tid * per + k;
+      if (e < trips * kRouteNW) loc += ceq[e];
+    }
+    int n_eq;
+    int run = block_exclusive_sum_512(loc, scan_ws, n_eq);
+    for (int k = 0; k < per; ++k) {
+      const int e = tid * per + k;
+      if (e < trips * kRouteNW) {
+        const int c = ceq[e];
+        ceq[e] = run;
+        run += c;
+      }
+    }
+    int n_gt;
+    block_exclusive_sum_512(gt, scan_ws, n_gt);
+    if (tid == 0) {
+      cnt2[0] = n_gt;
+      cnt2[1] = n_eq;
+    }
+  }
+  cl.sync();  // every chunk's counts are published
+  if (tid == 0) {
+    int sel_before = 0, eq_before = 0;
+    for (int r = 0; r < rank; ++r) {
+      const int* cr = cl.map_shared_rank(&cnt2[0], r);
+      const int r_gt = cr[0], r_eq = cr[1];
+      sel_before += r_gt + min(r_eq, max(0, need_eq - eq_before));
+      eq_before += r_eq;
+    }
+    sh_off[0] = n_route >= N ? c0 : (n_route <= 0 ? 0 : sel_before);
+    sh_off[1] = min(cnt2[1], max(0, need_eq - eq_before));  // equal keys of this chunk that are routed
+  }
+  __syncthreads();
+  const int sel_before = sh_off[0], take_eq = sh_off[1];
+  const unsigned lt = (1u << lane) - 1u;
+  auto selected = [&](int j, int i) -> bool {  // warp-collective
+    if (n_route <= 0) return false;
+    if (n_route >= N) return i < n;
+    const unsigned x = i < n ? rkeys[i] : 0u;
+    const bool eq = i < n && x == T;
+    const unsigned beq = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = ceq[j * kRouteNW + w] + __popc(beq & lt);
+    return i < n && (x > T || (eq && eq_rank < take_eq));
+  };
+  for (int j = 0; j < trips; ++j) {
+    const unsigned bal = __ballot_sync(0xffffffffu, selected(j, j * kRouteCT + tid));
+    if (lane == 0) csel[j * kRouteNW + w] = __popc(bal);
+  }
+  __syncthreads();
+  {
+    const int per = (trips * kRouteNW + kRouteCT - 1) / kRouteCT;
+    int loc = 0;
+    for (int k = 0; k < per; ++k) {
+      const int e = tid * per + k;
+      if (e < trips * kRouteNW) loc += csel[e];
+    }
+    int tot;
+    int run = block_exclusive_sum_512(loc, scan_ws, tot);
+    for (int k = 0; k < per; ++k) {
+      const int e = tid * per + k;
+      if (e < trips * kRouteNW) {
+        const int c = csel[e];
+        csel[e] = run;
+        run += c;
+      }
+    }
+    __syncthreads();
+  }
+  int32_t* rout = routed + static_cast<size_t>(bh) * n_route;
+  int32_t* tout = taylor + static_cast<size_t>(bh) * (N - n_route);
+  for (int j = 0; j < trips; ++j) {
+    const int i = j * kRouteCT + tid;
+    const bool sel = selected(j, i);
+    const unsigned bal = __ballot_sync(0xffffffffu, sel);
+    const int r = sel_before + csel[j * kRouteNW + w] + __popc(bal & lt);  // routed keys before c0 + i
+    if (i < n) {
+      // counts are exact by construction; the guards only keep a corrupted
+      // input (e.g. NaN sharpness) from writing past the buckets
+      const int gi = c0 + i;
+      if (sel) {
+        if (r < n_route) rout[r] = gi;
+        else if (status != nullptr) atomicCAS(status, 0, 1);
+      } else {
+        if (gi - r >= 0 && gi - r < N - n_route) tout[gi - r] = gi;
+        else if (status != nullptr) atomicCAS(status, 0, 1);
+      }
+    }
+  }
+  cl.sync();  // peers may still read this CTA's counts until here
+}
+
 cudaError_t launch_route(const float* sharp, int32_t* routed, int32_t* taylor, int BH, int N, int n_route,
                          int* status, cudaStream_t st) {
   if (BH <= 0 || N <= 0) return cudaSuccess;
+  cudaError_t e;
+  const int chunk = (N + kRouteCluster - 1) / kRouteCluster;
+  if (chunk <= kRouteChunkCap && static_cast<long long>(BH) * kRouteCluster <= 0x7fffffffLL) {
+    const int trips = (chunk + kRouteCT - 1) / kRouteCT;
+    const size_t smem = static_cast<size_t>(chunk) * 4 + static_cast<size_t>(2 * trips * kRouteNW) * 4;
+    e = cudaFuncSetAttribute(route_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem < 48 * 1024 ? 48 * 1024 : smem));
+    if (e != cudaSuccess) return e;
+    route_cluster_kernel<<<BH * kRouteCluster, kRouteCT, smem, st>>>(sharp, routed, taylor, N, n_route, status);
+    return cudaGetLastError();
+  }
   const size_t counts = static_cast<size_t>(route_count_words(N)) * 4;
   const size_t resident = static_cast<size_t>(N) * 4 + counts;
-  cudaError_t e;
   if (resident <= static_cast<size_t>(kRouteSmemBudget)) {
     e = cudaFuncSetAttribute(route_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouteSmemBudget);
     if (e != cudaSuccess) return e;
