@@ -100,6 +100,21 @@ def test_block_grouping_480p_sampled(cuda_ok):
         compare_head_blocks(cfg, bits, g, 0, h, rows=rows)
 
 
+def test_block_grouping_720p_two_heads(cuda_ok):
+    """Two of the 40 heads of the 720p latent workload (1182 query blocks per
+    head); sets whole, outputs on sampled rows."""
+    cfg = CONFIGS["720p"]
+    bits, (q, k, v) = inputs(cfg, heads=[0, 39])
+    sub = cfg.replace(H=2)
+    g = run_blocks(sub, q, k, v)
+    assert g["status"] == 0
+    rng = np.random.default_rng(19)
+    for h in range(2):
+        rows = np.unique(np.concatenate([rng.choice(cfg.N, 128, replace=False),
+                                         [0, cfg.N_src - 1, cfg.N_src, cfg.N - 1]]))
+        compare_head_blocks(sub, bits, g, 0, h, rows=rows)
+
+
 def test_padding_rows_are_never_stored(cuda_ok):
     """A row list with -1 entries only leaves out untouched and reports no
     error; an entry past N is reported."""

@@ -129,3 +129,18 @@ def test_taylor1_injected_timeout_is_reported(cuda_ok):
     again = api.isa_forward_taylor1(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws)
     assert api.isa_read_device_status(ws) == 0
     assert torch.equal(again.view(torch.int16), good.view(torch.int16))
+
+
+def test_taylor1_720p_two_heads(cuda_ok):
+    """Two of the 40 heads of the 720p latent workload (710 kept blocks: six
+    key tiles per item); C_b of every kept block and sampled output rows."""
+    cfg = CONFIGS["720p"]
+    bits, (q, k, v) = inputs(cfg, heads=[0, 39])
+    sub = cfg.replace(H=2)
+    g = run_t1(sub, q, k, v)
+    assert g["status"] == 0
+    rng = np.random.default_rng(17)
+    for h in range(2):
+        rows = np.unique(np.concatenate([rng.choice(cfg.N, 96, replace=False),
+                                         [0, cfg.N_src - 1, cfg.N_src, cfg.N - 1]]))
+        compare_head_t1(sub, bits, g, 0, h, rows=rows)
