@@ -45,7 +45,14 @@ Pins (see tests/test_oracle_pins.py): the saliency and sharpness formulas are
 readings, not printed by the pages ("parity unpinned" as to the pages); they
 are pinned by closed forms and by reduction to token-level attention computed
 with torch's scaled_dot_product_attention, which the pins use as an
-independent library routine.
+independent library routine.  The block-granular grouping (mean sharpness
+per query block) is a reading too ("parity unpinned" as to the pages),
+pinned by hand-worked means, rank counting, its reduction to per-token
+grouping at block = 1 and library attention
+(tests/test_oracle_block_route_pins.py).  The first-order Taylor variant
+follows from the expansion of exp around the block mean with no further
+reading; it is pinned by a per-token double loop, exact special cases and
+its second-order error scaling (tests/test_oracle_taylor1_pins.py).
 """
 from __future__ import annotations
 
