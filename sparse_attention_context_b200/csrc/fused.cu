@@ -20,11 +20,14 @@
 // while the current item computes, and the epilogue of one item overlaps the
 // QK^T products of the next: O goes from TMEM through registers into the
 // item's own Q buffer (free once its last QK^T is done) and leaves with one
-// TMA store per tile, so the softmax threads never wait on global stores.
+// TMA store per tile, issued by a warp of its own, so the softmax threads
+// neither issue stores nor wait for them.  The same warp loads the Q of
+// item k + 2 into that buffer as soon as the store has read it out, so the
+// K / V producer never waits on an output store.
 //
-// Warps (320 threads): 0-3 softmax of tile 0, 4-7 tile 1 (thread <-> query
+// Warps (352 threads): 0-3 softmax of tile 0, 4-7 tile 1 (thread <-> query
 // row <-> TMEM lane), 8 TMA producer, 9 TMEM allocator + the single UMMA
-// issuer.  TMEM: S/P of tile i at [128i, 128i + 128), O of tile i at
+// issuer, 10 Q loads and O stores (TMA) through the two Q buffers.  TMEM: S/P of tile i at [128i, 128i + 128), O of tile i at
 // [256 + D*i, 256 + D*i + D).  Tensor pipe order per key tile g (counted
 // across the CTA's items): PV0(g), S0(g+1), PV1(g), S1(g+1); S_i(g+1)
 // overwrites the P_i(g) columns PV_i(g) reads and is issued after it by the
@@ -51,20 +54,26 @@ struct FusedCfg {
   static constexpr int KT_BYTES = BN * D * 2;    // one key (or value) tile
   static constexpr int OFF_Q = 0;                // [buffer][tile]
   static constexpr int OFF_K = 4 * Q_BYTES;      // K hi, K lo
+  // K arrives and is released in 64-column chunks (hi chunks, then lo), the
+  // order in which the QK^T UMMAs read it: chunk j of key tile g+1 loads as
+  // soon as S_1(g) is done with chunk j, under S_1(g)'s later chunks and
+  // PV_0(g), instead of after the whole of S_1(g)
+  static constexpr int NKC = 2 * (D / 64);
+  static constexpr int KC_BYTES = BN * 128;      // one chunk: BN rows x 64 bf16
   static constexpr int OFF_V = OFF_K + 2 * KT_BYTES;
   static constexpr int OFF_BIAS = OFF_V + KT_BYTES;  // [2][BN] log2 cnt of key tiles g (ring by g & 1)
   static constexpr int OFF_BAR = OFF_BIAS + 2 * BN * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;
   static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
 struct FusedBars {
   uint64_t q_full[2][2];  // [buffer][tile]
-  uint64_t q_empty[2];    // buffer free: its O tiles stored out of it (one arrival per tile)
   uint64_t o_staged[2];   // O of tile i written into the staging buffer (128 arrivals)
-  uint64_t k_full, v_full, k_empty, v_empty;
+  uint64_t k_full[4], k_empty[4];  // per K chunk (hi c0, hi c1, lo c0, lo c1)
+  uint64_t v_full, v_empty;
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_done[2];
@@ -97,7 +106,7 @@ __device__ __forceinline__ void fregs_after(uint32_t (&r)[N]) {
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKhi,
                  const __grid_constant__ CUtensorMap tmKlo, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmO, const FlashParams p, int n_items) {
@@ -116,17 +125,26 @@ __global__ void __launch_bounds__(320, 1)
   const int my_items = n_items > static_cast<int>(blockIdx.x) ? (n_items - 1 - static_cast<int>(blockIdx.x)) / G + 1 : 0;
   const int nT = p.n_kv_tiles;
   const int total = my_items * nT;  // key tiles this CTA walks, over all its items
-  auto item_of = [&](int k) { return static_cast<int>(blockIdx.x) + k * G; };
+  // The CTAs' k-th items are consecutive in a head-minor order, so the ~148
+  // items in flight at once span every head (a few per head) instead of
+  // all being one head's: each head's Kbar / Vbar tiles are then read by a
+  // few SMs at a time, not by all of them from the same L2 lines.
+  const int n_heads = n_items / p.pairs_per_head;
+  auto item_of = [&](int k) {
+    const int lin = static_cast<int>(blockIdx.x) + k * G;
+    return (lin % n_heads) * p.pairs_per_head + lin / n_heads;
+  };
 
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->q_full[b][0], 1);
       mbar_init(&bars->q_full[b][1], 1);
-      mbar_init(&bars->q_empty[b], 2);
     }
-    mbar_init(&bars->k_full, 1);
+    for (int cc = 0; cc < 4; ++cc) {
+      mbar_init(&bars->k_full[cc], 1);
+      mbar_init(&bars->k_empty[cc], 1);
+    }
     mbar_init(&bars->v_full, 1);
-    mbar_init(&bars->k_empty, 1);
     mbar_init(&bars->v_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
@@ -159,53 +177,38 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
-      int q_issued = 0, g_issued = 0;
-      auto load_q = [&](int k) -> bool {
-        const int b = k & 1;
-        if (k >= 2 && !fw1(&bars->q_empty[b], ((k >> 1) - 1) & 1, bars, p)) return false;
-        const int item = item_of(k);
-        const int bh = item / p.pairs_per_head, row0 = (item % p.pairs_per_head) * 256;
-        for (int i = 0; i < 2; ++i) {
-          mbar_arrive_expect_tx(&bars->q_full[b][i], C::Q_BYTES);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(smem + C::OFF_Q + (b * 2 + i) * C::Q_BYTES + c * (128 * 128), &tmQ, &bars->q_full[b][i],
-                        c * 64, bh * p.N + row0 + i * 128);
-        }
-        q_issued = k + 1;
-        return true;
-      };
-      if (my_items > 0) ok = load_q(0);
+      int g_issued = 0;
       for (int g = 0; ok && g < total; ++g) {
         const int k = g / nT, t = g % nT;
         const int bh = item_of(k) / p.pairs_per_head;
         const int r = bh * p.kv_rows_per_head + t * BN;
-        if (g >= 1 && !(ok = fw1(&bars->k_empty, (g - 1) & 1, bars, p))) break;
-        mbar_arrive_expect_tx(&bars->k_full, 2 * C::KT_BYTES + BN * 4);
-        // key biases of tile g: slot g & 1 (the softmax of tile g-1 reads the
-        // other slot; it is done with slot g & 1 once S_1(g-1) has completed)
-        bulk_load(smem + C::OFF_BIAS + (g & 1) * BN * 4, p.bias2 + static_cast<size_t>(r), BN * 4, &bars->k_full);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_2d(smem + C::OFF_K + c * (BN * 128), &tmKhi, &bars->k_full, c * 64, r);
-          tma_load_2d(smem + C::OFF_K + C::KT_BYTES + c * (BN * 128), &tmKlo, &bars->k_full, c * 64, r);
+        for (int cc = 0; cc < C::NKC; ++cc) {
+          if (g >= 1 && !(ok = fw1(&bars->k_empty[cc], (g - 1) & 1, bars, p))) break;
+          const bool lo = cc >= D / 64;
+          const int c = lo ? cc - D / 64 : cc;
+          mbar_arrive_expect_tx(&bars->k_full[cc], C::KC_BYTES + (cc == 0 ? BN * 4 : 0));
+          // key biases of tile g ride with its first chunk: slot g & 1 (the
+          // softmax warps of tile g-2 read it, and both handed their P over
+          // before PV_1(g-2), which precedes S_1(g-1) in the tensor pipe)
+          if (cc == 0)
+            bulk_load(smem + C::OFF_BIAS + (g & 1) * BN * 4, p.bias2 + static_cast<size_t>(r), BN * 4,
+                      &bars->k_full[0]);
+          tma_load_2d(smem + C::OFF_K + (lo ? C::KT_BYTES : 0) + c * C::KC_BYTES, lo ? &tmKlo : &tmKhi,
+                      &bars->k_full[cc], c * 64, r);
         }
+        if (!ok) break;
         if (g >= 1 && !(ok = fw1(&bars->v_empty, (g - 1) & 1, bars, p))) break;
         mbar_arrive_expect_tx(&bars->v_full, C::KT_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) tma_load_2d(smem + C::OFF_V + c * (BN * 128), &tmV, &bars->v_full, c * 64, r);
         g_issued = g + 1;
-        // the next item's Q, as soon as its buffer is free (during this item)
-        if (t == 0 && k + 1 < my_items && !(ok = load_q(k + 1))) break;
       }
       // drain own copies still in flight
       if (g_issued > 0) {
-        mbar_wait_bounded(&bars->k_full, (g_issued - 1) & 1, nullptr, kWaitLimitNs);
+        for (int cc = 0; cc < C::NKC; ++cc)
+          mbar_wait_bounded(&bars->k_full[cc], (g_issued - 1) & 1, nullptr, kWaitLimitNs);
         mbar_wait_bounded(&bars->v_full, (g_issued - 1) & 1, nullptr, kWaitLimitNs);
-      }
-      for (int k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k) {
-        mbar_wait_bounded(&bars->q_full[k & 1][0], (k >> 1) & 1, nullptr, kWaitLimitNs);
-        mbar_wait_bounded(&bars->q_full[k & 1][1], (k >> 1) & 1, nullptr, kWaitLimitNs);
       }
     }
   } else if (warp == 9) {
@@ -214,20 +217,29 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t IDS = idesc_bf16(128, BN, 0);
       constexpr uint32_t IDO = idesc_bf16(128, D, 1);
       bool ok = true;
-      // S_i(g) = Q_i (hi + lo) of key tile g; commits s_full[i]
-      auto issue_S = [&](int i, int g) {
+      // S_i(g) = Q_i (hi + lo) of key tile g, chunk by chunk of K: S_0 waits
+      // for each chunk to land, S_1 (its last reader) releases each one;
+      // commits s_full[i] (false: a wait gave up)
+      auto issue_S = [&](int i, int g) -> bool {
         const int k = g / nT;
         const uint32_t qa = aQ + ((k & 1) * 2 + i) * C::Q_BYTES;
         const uint32_t dS = tmem + i * BN;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
-                    desc_k_sw128(aK + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, kk > 0 ? 1u : 0u);
+        for (int cc = 0; cc < C::NKC; ++cc) {
+          const int c = cc % (D / 64);
+          const uint32_t kb = aK + (cc >= D / 64 ? C::KT_BYTES : 0) + c * C::KC_BYTES;
+          if (i == 0) {
+            if (!fw1(&bars->k_full[cc], g & 1, bars, p)) return false;
+            tc_fence_after();
+          }
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16(dS, desc_k_sw128(qa + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
-                    desc_k_sw128(aK + C::KT_BYTES + (kk >> 2) * (BN * 128) + (kk & 3) * 32), IDS, 1u);
+          for (int k4 = 0; k4 < 4; ++k4)
+            umma_bf16(dS, desc_k_sw128(qa + c * (128 * 128) + k4 * 32), desc_k_sw128(kb + k4 * 32), IDS,
+                      (cc > 0 || k4 > 0) ? 1u : 0u);
+          if (i == 1) umma_commit(&bars->k_empty[cc]);
+        }
         umma_commit(&bars->s_full[i]);
+        return true;
       };
       // waits for the Q of key tile g's item (first tile of an item only)
       auto q_ready = [&](int g) -> bool {
@@ -248,33 +260,60 @@ __global__ void __launch_bounds__(320, 1)
         umma_commit(&bars->o_done[i]);
         return true;
       };
-      if (total > 0) {
-        ok = q_ready(0) && fw1(&bars->k_full, 0, bars, p);
-        if (ok) {
-          tc_fence_after();
-          issue_S(0, 0);
-          issue_S(1, 0);
-          umma_commit(&bars->k_empty);
-        }
-      }
+      if (total > 0) ok = q_ready(0) && issue_S(0, 0) && issue_S(1, 0);
       for (int g = 0; ok && g < total; ++g) {
         const bool more = g + 1 < total;
         if (!(ok = fw1(&bars->v_full, g & 1, bars, p))) break;
         if (!(ok = issue_PV(0, g))) break;
-        if (more) {
-          if (!(ok = q_ready(g + 1) && fw1(&bars->k_full, (g + 1) & 1, bars, p))) break;
-          tc_fence_after();
-          issue_S(0, g + 1);
-        }
+        if (more && !(ok = q_ready(g + 1) && issue_S(0, g + 1))) break;
         if (!(ok = issue_PV(1, g))) break;
         umma_commit(&bars->v_empty);
-        if (more) {
-          issue_S(1, g + 1);
-          umma_commit(&bars->k_empty);
-        }
+        if (more && !(ok = issue_S(1, g + 1))) break;
       }
       umma_commit(&bars->teardown);
       mbar_wait_bounded(&bars->teardown, 0, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == 10) {
+    // ---------------------------------- Q loads and O stores of each item
+    if (lane == 0) {
+      int q_issued = 0;
+      auto load_q = [&](int k) {  // Q of item k into buffer k & 1
+        const int b = k & 1;
+        const int item = item_of(k);
+        const int bh = item / p.pairs_per_head, row0 = (item % p.pairs_per_head) * 256;
+        for (int i = 0; i < 2; ++i) {
+          mbar_arrive_expect_tx(&bars->q_full[b][i], C::Q_BYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(smem + C::OFF_Q + (b * 2 + i) * C::Q_BYTES + c * (128 * 128), &tmQ, &bars->q_full[b][i],
+                        c * 64, bh * p.N + row0 + i * 128);
+        }
+        q_issued = k + 1;
+      };
+      for (int k = 0; k < 2 && k < my_items; ++k) load_q(k);
+      for (int k = 0; k < my_items; ++k) {
+        const int item = item_of(k);
+        const int bh = item / p.pairs_per_head, b = k & 1;
+        bool ok = true;
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (!(ok = fw1(&bars->o_staged[i], k & 1, bars, p))) break;
+          const int row0 = (item % p.pairs_per_head) * 256 + i * 128;
+          uint8_t* stage = smem + C::OFF_Q + (b * 2 + i) * C::Q_BYTES;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) tma_store_3d(&tmO, stage + c * (128 * 128), c * 64, row0, bh);
+        }
+        bulk_commit_group();
+        if (!ok) break;
+        if (k + 2 < my_items) {
+          bulk_wait_read_all();  // buffer b is free once the stores have read it
+          load_q(k + 2);
+        }
+      }
+      bulk_wait_all();  // stores complete before the CTA ends
+      for (int k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k) {  // and own loads (error paths)
+        mbar_wait_bounded(&bars->q_full[k & 1][0], (k >> 1) & 1, nullptr, kWaitLimitNs);
+        mbar_wait_bounded(&bars->q_full[k & 1][1], (k >> 1) & 1, nullptr, kWaitLimitNs);
+      }
     }
   } else {
     // ------------------------------------------ softmax warpgroup of tile i
@@ -386,25 +425,27 @@ __global__ void __launch_bounds__(320, 1)
       // epilogue of item k: sharpness and Taylor output of this row.  O_i
       // leaves TMEM through registers into Q buffer k & 1 (its last QK^T,
       // S_1 of the item's last key tile, completed before PV_0 of that tile
-      // did, hence before o_done) in the TMA box layout, and one thread of
-      // the warpgroup stores the tile; rows past N are clipped by the map.
+      // did, hence before o_done) in the TMA box layout; the store warp
+      // sends the tile out (rows past N are clipped by the map).
       if (!(ok = fwarp(&bars->o_done[i], (k * nT + nT - 1) & 1, bars, p))) break;
       tc_fence_after();
       const int b = k & 1;
       uint8_t* stage = smem + C::OFF_Q + (b * 2 + i) * C::Q_BYTES;
       const float inv = 1.f / l;
       if (g_row < p.n_rows) p.sharp[static_cast<size_t>(bh) * p.N + g_row] = ex2(mx - m) * inv;  // max_b softmax_b
+      // all of O_i in flight at once, one wait; then the next item's first
+      // PV may overwrite it
+      uint32_t ou[D / 32][32];
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) tmem_ld32(sO + j * 32, ou[j]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) fregs_after(ou[j]);
+      tc_fence_before();
+      mbar_arrive(&bars->o_free[i]);
 #pragma unroll
       for (int j = 0; j < D / 32; ++j) {
-        uint32_t u[32];
-        tmem_ld32(sO + j * 32, u);
-        tmem_wait_ld();
-        fregs_after(u);
-        if (j == D / 32 - 1) {
-          // O of this tile is in registers: the next item's first PV may overwrite it
-          tc_fence_before();
-          mbar_arrive(&bars->o_free[i]);
-        }
+        const uint32_t (&u)[32] = ou[j];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const uint32_t x = pack_bf16(__uint_as_float(u[8 * q4 + 0]) * inv, __uint_as_float(u[8 * q4 + 1]) * inv);
@@ -417,22 +458,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       fence_proxy_async_smem();  // the generic-proxy writes above, for the TMA store
       mbar_arrive(&bars->o_staged[i]);
-      if ((warp & 3) == 0 && lane == 0) {
-        if (fw1(&bars->o_staged[i], k & 1, bars, p)) {
-          const int row0 = (item % p.pairs_per_head) * 256 + i * 128;
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) tma_store_3d(&tmO, stage + c * (128 * 128), c * 64, row0, bh);
-          bulk_commit_group();
-          bulk_wait_read_all();  // the staging buffer may be reloaded with Q once read
-          mbar_arrive(&bars->q_empty[b]);
-        } else {
-          ok = false;
-        }
-      }
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
     }
-    if ((warp & 3) == 0 && lane == 0) bulk_wait_all();  // stores complete before the CTA ends
   }
 
   tc_fence_before();
