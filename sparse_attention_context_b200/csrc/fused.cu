@@ -109,7 +109,7 @@ template <int D>
 __global__ void __launch_bounds__(352, 1)
     fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKhi,
                  const __grid_constant__ CUtensorMap tmKlo, const __grid_constant__ CUtensorMap tmV,
-                 const __grid_constant__ CUtensorMap tmO, const FlashParams p, int n_items) {
+                 const __grid_constant__ CUtensorMap tmO, const FlashParams p, int n_items, int n_heads) {
   using C = FusedCfg<D>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -129,7 +129,6 @@ __global__ void __launch_bounds__(352, 1)
   // items in flight at once span every head (a few per head) instead of
   // all being one head's: each head's Kbar / Vbar tiles are then read by a
   // few SMs at a time, not by all of them from the same L2 lines.
-  const int n_heads = n_items / p.pairs_per_head;
   auto item_of = [&](int k) {
     const int lin = static_cast<int>(blockIdx.x) + k * G;
     return (lin % n_heads) * p.pairs_per_head + lin / n_heads;
@@ -487,14 +486,14 @@ cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi
     if ((e = cudaFuncSetAttribute(fused_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)) !=
         cudaSuccess)
       return e;
-    fused_kernel<128><<<grid, C::THREADS, C::SMEM, st>>>(tmQ, tmKhi, tmKlo, tmV, tmO, p, static_cast<int>(items));
+    fused_kernel<128><<<grid, C::THREADS, C::SMEM, st>>>(tmQ, tmKhi, tmKlo, tmV, tmO, p, static_cast<int>(items), BH);
   } else if (D == 64) {
     using C = FusedCfg<64>;
     const int smem = C::SMEM < 116 * 1024 ? 116 * 1024 : C::SMEM;  // one CTA per SM (all 512 TMEM columns)
     if ((e = cudaFuncSetAttribute(fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return e;
-    fused_kernel<64><<<grid, C::THREADS, smem, st>>>(tmQ, tmKhi, tmKlo, tmV, tmO, p, static_cast<int>(items));
+    fused_kernel<64><<<grid, C::THREADS, smem, st>>>(tmQ, tmKhi, tmKlo, tmV, tmO, p, static_cast<int>(items), BH);
   } else {
     return cudaErrorInvalidValue;
   }
