@@ -547,7 +547,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="isa", choices=["isa", "reference"])
     ap.add_argument("--config", default="480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
