@@ -2,11 +2,11 @@
 4 in every channel and a few keys to 2 or 4 in every channel, so those rows'
 largest score jumps by 90-260 (base-2 units) in a later key tile: in the
 first or the second half of a tile, once or twice, in the ragged last tile,
-for some rows of a warp and not the others.  Such rows leave the engine's
-speculative exponent pass (which starts on the previous tile's reference)
-for its recomputation on the new reference, with O and l rescaled; their
-outputs must still match the float64 oracle, in the dense engine and in the
-full attention of ISA (128- and 64-key tiles)."""
+for some rows of a warp and not the others.  Such rows move the engine's
+running reference past its 2^32 threshold, so O and l are rescaled by
+2^(m_old - m_new) mid-sequence (by some warps of a tile and not others);
+their outputs must still match the float64 oracle, in the dense engine and
+in the full attention of ISA (128- and 64-key tiles)."""
 import numpy as np
 import pytest
 
