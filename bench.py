@@ -53,8 +53,11 @@ def counts(cfg):
 
     nSB = -(-cfg.N_src // cfg.block)
     nCB = -(-cfg.N_ctx // cfg.block)
-    n_keep = int(min(max(math.ceil(cfg.keep * nCB - 1e-6 * nCB), 0), nCB))
-    n_route = int(min(max(math.ceil(cfg.rho * cfg.N - 1e-6 * cfg.N), 0), cfg.N))
+    def guarded(frac, n):  # ceil(frac*n - min(1e-6*n, 0.5)) in [0, n], as the library counts
+        return int(min(max(math.ceil(frac * n - min(1e-6 * n, 0.5)), 0), n))
+
+    n_keep = guarded(cfg.keep, nCB)
+    n_route = guarded(cfg.rho, cfg.N)
     return nSB, nCB, n_keep, n_route
 
 

@@ -17,9 +17,10 @@
  *   s        scale (1/sqrt(d) when shape->scale <= 0).
  *   saliency sal_c = sum_r cnt_r * softmax_c(s Qbar_r.Kbar_c + ln cnt_c) / N
  *            over all key blocks c; context blocks ranked by it; the top
- *            n_keep = ceil(keep*nCB - 1e-6*nCB) are kept; source blocks always.
+ *            n_keep = ceil(keep*nCB - g(nCB)) are kept; source blocks always;
+ *            g(n) = min(1e-6*n, 0.5) absorbs the float32 rounding of keep/rho.
  *   sharp_i  max_b softmax_b(s q_i.Kbar_b + ln cnt_b) over kept blocks.
- *   routing  the n_route = ceil(rho*N - 1e-6*N) sharpest queries (ties: lower
+ *   routing  the n_route = ceil(rho*N - g(N)) sharpest queries (ties: lower
  *            index first) -> full attention over every token of every kept
  *            block; the others -> sum_b cnt_b e^{s q.Kbar_b} Vbar_b /
  *            sum_b cnt_b e^{s q.Kbar_b} over kept blocks.
@@ -71,15 +72,15 @@ typedef struct {
   float keep, rho, scale;
 } isa_shape;
 
-/* Number of kept context blocks per (b, h): ceil(keep*nCB - 1e-6*nCB), nCB =
+/* Number of kept context blocks per (b, h): ceil(keep*nCB - g(nCB)), nCB =
  * ceil(N_ctx/block).  Returns -1 on an invalid shape. */
 int isa_n_keep(const isa_shape* shape);
 
-/* Number of routed queries per (b, h): ceil(rho*N - 1e-6*N).  -1 if invalid. */
+/* Number of routed queries per (b, h): ceil(rho*N - g(N)).  -1 if invalid. */
 int isa_n_route(const isa_shape* shape);
 
 /* Number of routed query blocks per (b, h) of the block-granular grouping
- * (isa_route_blocks_taylor_fwd): ceil(rho*nB - 1e-6*nB), nB = nSB + nCB.
+ * (isa_route_blocks_taylor_fwd): ceil(rho*nB - g(nB)), nB = nSB + nCB.
  * -1 if invalid. */
 int isa_n_route_blocks(const isa_shape* shape);
 

@@ -24,10 +24,11 @@ The exact formulas below are the plainest reading of that outline:
 * saliency of key block c: mean over query blocks r (weighted by cnt_r) of
   the block-level attention softmax_c( s * Qbar_r . Kbar_c + ln cnt_c ),
   over all key blocks; context blocks are ranked by it and the top
-  n_keep = ceil(keep*nCB - 1e-6*nCB) are kept, all source blocks always kept;
+  n_keep = ceil(keep*nCB - g(nCB)) are kept, all source blocks always kept,
+  with the guard g(n) = min(1e-6*n, 0.5) (see ``guarded_count``);
 * sharpness of query i: the largest probability of the block-level
   distribution softmax_b( s * q_i . Kbar_b + ln cnt_b ) over kept blocks;
-* routing: the n_route = ceil(rho*N - 1e-6*N) sharpest queries get full
+* routing: the n_route = ceil(rho*N - g(N)) sharpest queries get full
   attention over every kept token; ties rank the lower index first;
 * 0-th order Taylor attention: exp(s q.k_j) is replaced by exp(s q.Kbar_b)
   for every j in block b, in numerator and denominator; summing over the
@@ -38,7 +39,7 @@ The exact formulas below are the plainest reading of that outline:
   to the numerator, C_b = sum_{j in b} (k_j - Kbar_b) v_j^T;
 * variant grouping by whole query blocks (``granularity="block"``): a query
   block (same per-segment partition as the keys) scores the mean sharpness
-  of its queries, and the n_route_blocks = ceil(rho*nB - 1e-6*nB) best
+  of its queries, and the n_route_blocks = ceil(rho*nB - g(nB)) best
   blocks (ties: lower block index) are routed whole.
 
 Pins (see tests/test_oracle_pins.py): the saliency and sharpness formulas are
@@ -67,19 +68,27 @@ NEG_INF = -np.inf
 # Counts and block layout
 # ---------------------------------------------------------------------------
 
-def n_keep_of(keep: float, nCB: int) -> int:
-    """Number of context blocks kept: ceil(keep*nCB - 1e-6*nCB) in [0, nCB].
+def guarded_count(frac: float, n: int) -> int:
+    """ceil(frac*n - g) clamped to [0, n], with the guard g = min(1e-6*n, 0.5).
 
-    The relative guard keeps exact products such as 0.25*256 from rounding up
-    when the fraction arrives as a float32 (0.25f*256 is exact, 0.2f*40560
-    is 8112.0001).
+    The fractions keep and rho reach the kernels as float32, whose rounding
+    moves frac*n by up to 6e-8*n (0.2f*40560 = 8112.0001 must count 8112).
+    The guard 1e-6*n absorbs that; it is capped at one half so that an exact
+    integral product never loses a unit (at n >= 10^6 the uncapped guard
+    would count 200001 for 0.200002 * 10^6).  A genuinely fractional product
+    whose fraction is within the guard rounds down.
     """
-    return int(min(max(math.ceil(keep * nCB - 1e-6 * nCB), 0), nCB))
+    return int(min(max(math.ceil(frac * n - min(1e-6 * n, 0.5)), 0), n))
+
+
+def n_keep_of(keep: float, nCB: int) -> int:
+    """Number of context blocks kept: ceil(keep*nCB - g(nCB)) in [0, nCB]."""
+    return guarded_count(keep, nCB)
 
 
 def n_route_of(rho: float, N: int) -> int:
-    """Number of queries routed to full attention: ceil(rho*N - 1e-6*N) in [0, N]."""
-    return int(min(max(math.ceil(rho * N - 1e-6 * N), 0), N))
+    """Number of queries routed to full attention: ceil(rho*N - g(N)) in [0, N]."""
+    return guarded_count(rho, N)
 
 
 def block_layout(N_src: int, N_ctx: int, blk: int):
@@ -182,8 +191,8 @@ def sharpness(q, Kbar_K, cnt_K, scale):
 # ---------------------------------------------------------------------------
 
 def n_route_blocks_of(rho: float, nB: int) -> int:
-    """Number of query blocks routed to full attention: ceil(rho*nB - 1e-6*nB) in [0, nB]."""
-    return int(min(max(math.ceil(rho * nB - 1e-6 * nB), 0), nB))
+    """Number of query blocks routed to full attention: ceil(rho*nB - g(nB)) in [0, nB]."""
+    return guarded_count(rho, nB)
 
 
 def block_mean_sharpness(sharp, starts, cnts):

@@ -40,14 +40,16 @@ int split_ctas_for_device() {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-int keep_count(float keep, int nCB) {
-  const double v = std::ceil(static_cast<double>(keep) * nCB - 1e-6 * nCB);
-  return static_cast<int>(std::min<double>(std::max<double>(v, 0.0), nCB));
+// ceil(frac*n - g) in [0, n], guard g = min(1e-6*n, 0.5): absorbs the float32
+// rounding of frac (0.2f*40560 = 8112.0001 counts 8112) and never takes a
+// whole unit off an exact product.
+int guarded_count(float frac, int n) {
+  const double g = std::min(1e-6 * n, 0.5);
+  const double v = std::ceil(static_cast<double>(frac) * n - g);
+  return static_cast<int>(std::min<double>(std::max<double>(v, 0.0), n));
 }
-int route_count(float rho, int N) {
-  const double v = std::ceil(static_cast<double>(rho) * N - 1e-6 * N);
-  return static_cast<int>(std::min<double>(std::max<double>(v, 0.0), N));
-}
+int keep_count(float keep, int nCB) { return guarded_count(keep, nCB); }
+int route_count(float rho, int N) { return guarded_count(rho, N); }
 
 int check_shape(const isa_shape* s, Dims* o) {
   if (s == nullptr) return ISA_ERR_INVALID_ARG;

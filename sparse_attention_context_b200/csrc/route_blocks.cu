@@ -5,7 +5,7 @@
 // queries) are grouped for full attention.  The abstract does not fix the
 // unit that is grouped; this variant groups the per-segment token blocks
 // that the keys already use: a query block scores the mean sharpness of its
-// cnt_b queries, and the n_rb = ceil(rho*nB - 1e-6*nB) best blocks (ties:
+// cnt_b queries, and the n_rb = ceil(rho*nB - min(1e-6*nB, 0.5)) best blocks (ties:
 // lower block index first) are routed whole.  A routed group is then a run
 // of consecutive rows, so full attention needs no scattered query set.
 //

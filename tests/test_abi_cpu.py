@@ -49,7 +49,9 @@ def shape(**kw):
 
 @pytest.mark.parametrize("keep,rho,N_src,N_ctx,blk", [
     (0.25, 0.2, 20280, 20280, 128), (0.5, 0.25, 256, 256, 64), (0.3, 0.2, 4096, 4096, 128),
-    (0.2, 0.15, 75600, 75600, 128), (0.0, 0.0, 100, 0, 64), (1.0, 1.0, 77, 300, 64), (0.1, 0.5, 32768, 32768, 128)])
+    (0.2, 0.15, 75600, 75600, 128), (0.0, 0.0, 100, 0, 64), (1.0, 1.0, 77, 300, 64), (0.1, 0.5, 32768, 32768, 128),
+    # the guard's cap: 0.200002 * 10^6 is an exact count at N >= 10^6
+    (0.5, 0.200002, 600000, 400000, 128), (0.5, 1.0, 1900000, 100000, 128)])
 def test_counts_match_oracle(L, keep, rho, N_src, N_ctx, blk):
     s = shape(N_src=N_src, N_ctx=N_ctx, block=blk, keep=keep, rho=rho)
     nCB = -(-N_ctx // blk)

@@ -51,7 +51,7 @@ def test_block_route_matches_rank_counting(seed):
             if ahead < nrb:
                 sel.append(b)
         assert blocks.tolist() == sel
-        assert len(sel) == nrb == int(np.ceil(rho * nB - 1e-6 * nB))
+        assert len(sel) == nrb == int(np.ceil(rho * nB - min(1e-6 * nB, 0.5)))
 
 
 def test_block_route_with_one_token_blocks_is_token_route():

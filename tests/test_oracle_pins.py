@@ -261,3 +261,97 @@ def test_context_less_salient_than_source(name):
     r = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     nSB = r["nSB"]
     assert r["sal_all"][nSB:].mean() < r["sal_all"][:nSB].mean()
+
+
+# ------------------------------------------------------------ k-th value
+def test_kth_value_hand_worked():
+    """kth_value sets the tie window of every set comparison, so it is pinned
+    by exact values: descending order 0.9, 0.9, 0.5, 0.3, 0.1."""
+    s = np.array([0.3, 0.9, 0.1, 0.9, 0.5])
+    assert oracle.kth_value(s, 0) == math.inf
+    assert oracle.kth_value(s, 1) == 0.9
+    assert oracle.kth_value(s, 2) == 0.9          # a tie with the first
+    assert oracle.kth_value(s, 3) == 0.5          # the (k+1)-th value would be 0.3
+    assert oracle.kth_value(s, 4) == 0.3
+    assert oracle.kth_value(s, 5) == 0.1          # k = len: the smallest score
+    assert oracle.kth_value(np.array([2.0]), 1) == 2.0
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_kth_value_is_the_order_statistic(seed):
+    """Brute-force definition of the k-th largest value t: fewer than k scores
+    lie strictly above t and at least k lie at or above it, and t is one of
+    the scores; it is also the smallest score of the top-k set."""
+    rng = np.random.default_rng(seed)
+    s = rng.integers(0, 7, size=23).astype(np.float64) / 7.0  # many ties
+    for k in range(1, 24):
+        t = oracle.kth_value(s, k)
+        assert t in s
+        assert np.sum(s > t) < k <= np.sum(s >= t)
+        assert t == s[oracle.topk_ascending(s, k)].min()
+
+
+# ------------------------------------------------------------ count guard
+def test_count_guard_hand_worked():
+    """Counts are ceil(frac*n - g) with g = min(1e-6*n, 0.5) (a reading: keep
+    and rho reach the kernels as float32, whose rounding moves frac*n by up to
+    6e-8*n).  Hand-worked cases on both sides of the guard:
+      rho = 0.2 as float32 (0.20000000298...), N = 40560: 8112.00012 -> 8112
+        (a plain ceiling would give 8113);
+      rho = 0.2000101, N = 40560: 8112.41, guard 0.0406 -> 8113;
+      rho = 0.2000005, N = 10^6: 200000.5, guard 0.5 (capped) -> 200000;
+      rho = 0.200002, N = 10^6: 200002 exactly -> 200002 (an uncapped guard of
+        1.0 would give 200001);
+      rho = 1, N = 2*10^7: all rows;
+      keep = 0.3f, nCB = 32: 9.6000001 -> 10;  keep = 0.25f, nCB = 159: 39.75 -> 40."""
+    assert oracle.n_route_of(float(np.float32(0.2)), 40560) == 8112
+    assert oracle.n_route_of(0.2000101, 40560) == 8113
+    assert oracle.n_route_of(0.2000005, 1_000_000) == 200000
+    assert oracle.n_route_of(0.200002, 1_000_000) == 200002
+    assert oracle.n_route_of(1.0, 20_000_000) == 20_000_000
+    assert oracle.n_keep_of(float(np.float32(0.3)), 32) == 10
+    assert oracle.n_keep_of(float(np.float32(0.25)), 159) == 40
+    assert oracle.guarded_count(0.5, 7) == 4 and oracle.guarded_count(0.0, 7) == 0
+
+
+# ------------------------------------------------------- batched entry points
+def test_dense_equals_library_over_batch_and_heads():
+    """oracle.dense over [B, H, N, d] against torch SDPA (float64), with
+    distinct heads so that a swapped or dropped (b, h) index fails."""
+    rng = np.random.default_rng(30)
+    q, k, v = (rng.standard_normal((2, 3, 70, 16)) for _ in range(3))
+    q[1, 2] *= 3.0
+    ref = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(x) for x in (q, k, v))).numpy()
+    assert np.allclose(oracle.dense(q, k, v), ref, rtol=1e-10, atol=1e-12)
+    ref2 = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(x) for x in (q, k, v)),
+                                                            scale=0.3).numpy()
+    assert np.allclose(oracle.dense(q, k, v, scale=0.3), ref2, rtol=1e-10, atol=1e-12)
+
+
+def test_isa_fwd_keep1_rho1_equals_library_dense_over_batch():
+    """keep = rho = 1: the batched forward is dense attention for every (b, h)."""
+    rng = np.random.default_rng(31)
+    q, k, v = (rng.standard_normal((2, 2, 150, 16)) for _ in range(3))
+    ref = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(x) for x in (q, k, v))).numpy()
+    assert np.allclose(oracle.isa_fwd(q, k, v, 90, 32, 1.0, 1.0), ref, rtol=1e-10, atol=1e-12)
+
+
+def test_isa_fwd_rho0_equals_library_on_replaced_keys_per_head():
+    """rho = 0, keep < 1: every row of every (b, h) is Taylor attention, which
+    is library attention over the kept tokens with each key replaced by its
+    block mean (values per token).  The kept set is taken per head from
+    isa_head, the output from isa_fwd, the reference from SDPA."""
+    rng = np.random.default_rng(32)
+    B, H, N_src, N_ctx, blk, d = 2, 2, 100, 90, 32, 8
+    q, k, v = (rng.standard_normal((B, H, N_src + N_ctx, d)) for _ in range(3))
+    k[:, :, N_src:] *= 0.5
+    out = oracle.isa_fwd(q, k, v, N_src, blk, 0.5, 0.0)
+    starts, cnts = oracle.block_layout(N_src, N_ctx, blk)[:2]
+    for b in range(B):
+        for h in range(H):
+            r = oracle.isa_head(q[b, h], k[b, h], v[b, h], N_src, blk, 0.5, 0.0)
+            k_rep = np.empty_like(k[b, h])
+            for s, c in zip(starts, cnts):
+                k_rep[s:s + c] = k[b, h, s:s + c].mean(axis=0)
+            T = r["tokens"]
+            assert np.allclose(out[b, h], sdpa(q[b, h], k_rep[T], v[b, h, T]), rtol=1e-10, atol=1e-12)
