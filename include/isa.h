@@ -42,7 +42,9 @@
  *   isa_status; on an error nothing is launched.  Launches are asynchronous
  *   on `stream` (a cudaStream_t; NULL = legacy default stream).  A kernel
  *   that gives up on a bounded wait writes ISA_ERR_DEVICE_TIMEOUT into the
- *   status word and exits; read it with isa_read_device_status().
+ *   status word and exits; read it with isa_read_device_status().  After a
+ *   non-zero device status the outputs of the calls since the last reset
+ *   are undefined (rows may be left unwritten).
  * - Supported: d in {64, 128}; block in {64, 128}; N_src >= 1; N_ctx >= 0;
  *   0 <= keep <= 1; 0 <= rho <= 1; ceil(N_ctx/block) <= 4096;
  *   B*H <= 65535.  Anything else returns ISA_ERR_UNSUPPORTED.
@@ -234,8 +236,9 @@ int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, co
  * one array, which keeps the last call's contents: calls that overlap on
  * the GPU (different streams, or different host threads on one device)
  * race and corrupt each other.  The device status word of these calls is
- * not readable by the caller; use isa_forward with an own workspace when
- * device-side timeouts must be observed. */
+ * not readable by the caller, so a device-side timeout (which leaves rows of
+ * out unwritten or stale) goes unseen here; use isa_forward with an own
+ * workspace when device-side timeouts must be observed. */
 #define ISA_STATIC_SCRATCH_BYTES (64u << 20)
 int isa_forward_static(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                        uint16_t* out, void* stream);

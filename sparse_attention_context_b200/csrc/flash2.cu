@@ -539,6 +539,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rr_all = blockIdx.x * 8 + warp;
   if (rr_all >= n_items * 256) return;
+  // A piece that gave up on a bounded wait wrote no partials: leave the rows
+  // unwritten rather than merge whatever the buffers held before.
+  if (p.status != nullptr && *reinterpret_cast<const volatile int*>(p.status) != 0) return;
   const int s = rr_all / 256, rr = rr_all % 256;
   const int item = item_base + s;
   const int bh = item / p.pairs_per_head;

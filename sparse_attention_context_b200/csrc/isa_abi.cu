@@ -7,6 +7,8 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "isa.h"
@@ -130,13 +132,7 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
   return ISA_OK;
 }
 
-thread_local cudaError_t g_last_cuda_error = cudaSuccess;  // reported by isa_last_error()
-
-int cuda_status(cudaError_t e) {
-  if (e == cudaSuccess) return ISA_OK;
-  g_last_cuda_error = e;
-  return ISA_ERR_CUDA;
-}
+int cuda_status(cudaError_t e) { return record_cuda_status(e); }
 
 // --- tensor maps (driver entry point fetched once through the runtime)
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -388,6 +384,22 @@ bool tensors_ok(std::initializer_list<const void*> ps) {
 
 }  // namespace
 
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;  // reported by isa_last_error()
+
+bool nvtx_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("ISA_NVTX");
+    return e != nullptr && e[0] != '\0' && std::strcmp(e, "0") != 0;
+  }();
+  return on;
+}
+
+int record_cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ISA_OK;
+  g_last_cuda_error = e;
+  return ISA_ERR_CUDA;
+}
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
@@ -441,6 +453,7 @@ size_t isa_workspace_size(const isa_shape* shape) {
 
 int isa_preselect_ctx(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                       int32_t* kept_ctx_idx, float* saliency, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_preselect_ctx");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -452,6 +465,7 @@ int isa_preselect_ctx(const isa_shape* shape, const uint16_t* q, const uint16_t*
 
 int isa_route_queries(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx, int32_t* routed_idx,
                       int32_t* taylor_idx, float* sharpness, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_route_queries");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -466,6 +480,7 @@ int isa_route_queries(const isa_shape* shape, const uint16_t* q, const int32_t* 
 int isa_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                  const int32_t* kept_ctx_idx, const int32_t* routed_idx, const int32_t* taylor_idx, uint16_t* out,
                  void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_attn_fwd");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -479,6 +494,7 @@ int isa_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, c
 int isa_route_taylor_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
                          int32_t* routed_idx, int32_t* taylor_idx, float* sharpness, uint16_t* out, void* ws,
                          size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_route_taylor_fwd");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -493,6 +509,7 @@ int isa_route_taylor_fwd(const isa_shape* shape, const uint16_t* q, const int32_
 int isa_full_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                       const int32_t* kept_ctx_idx, const int32_t* routed_idx, uint16_t* out, void* ws,
                       size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_full_attn_fwd");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -504,6 +521,7 @@ int isa_full_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t*
 
 int isa_taylor_attn_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
                         const int32_t* taylor_idx, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_taylor_attn_fwd");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -515,6 +533,7 @@ int isa_taylor_attn_fwd(const isa_shape* shape, const uint16_t* q, const int32_t
 
 int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                 void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_forward");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -522,15 +541,25 @@ int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, co
   int32_t* kept = at<int32_t>(ws, c.L.kept);
   int32_t* routed = at<int32_t>(ws, c.L.routed);
   int32_t* taylor = at<int32_t>(ws, c.L.taylor);
-  rc = run_preselect(c, q, k, v, kept, nullptr);
-  if (rc == ISA_OK) rc = run_route_taylor(c, q, kept, routed, taylor, nullptr, out);
-  if (rc == ISA_OK) rc = run_full(c, q, k, v, kept, routed, out);
+  {
+    NvtxRange r("isa_forward: pre-selection");
+    rc = run_preselect(c, q, k, v, kept, nullptr);
+  }
+  if (rc == ISA_OK) {
+    NvtxRange r("isa_forward: sharpness + Taylor + route");
+    rc = run_route_taylor(c, q, kept, routed, taylor, nullptr, out);
+  }
+  if (rc == ISA_OK) {
+    NvtxRange r("isa_forward: full attention");
+    rc = run_full(c, q, k, v, kept, routed, out);
+  }
   return rc;
 }
 
 int isa_route_blocks_taylor_fwd(const isa_shape* shape, const uint16_t* q, const int32_t* kept_ctx_idx,
                                 int32_t* routed_blk_idx, int32_t* routed_rows, float* block_score, float* sharpness,
                                 uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_route_blocks_taylor_fwd");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -546,6 +575,7 @@ int isa_route_blocks_taylor_fwd(const isa_shape* shape, const uint16_t* q, const
 int isa_full_attn_rows_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                            const int32_t* kept_ctx_idx, const int32_t* row_idx, int n_rows, uint16_t* out,
                            void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_full_attn_rows_fwd");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -559,6 +589,7 @@ int isa_full_attn_rows_fwd(const isa_shape* shape, const uint16_t* q, const uint
 
 int isa_forward_blocks(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                        uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_forward_blocks");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -582,6 +613,7 @@ size_t isa_taylor1_workspace_size(const isa_shape* shape) {
 int isa_taylor1_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                          const int32_t* kept_ctx_idx, const int32_t* taylor_idx, uint16_t* out, void* ws,
                          size_t ws_bytes, void* cws, size_t cws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_taylor1_attn_fwd");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -598,6 +630,7 @@ int isa_taylor1_attn_fwd(const isa_shape* shape, const uint16_t* q, const uint16
 
 int isa_forward_taylor1(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         uint16_t* out, void* ws, size_t ws_bytes, void* cws, size_t cws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_forward_taylor1");
   Ctx c;
   int rc = make_ctx(shape, ws, ws_bytes, stream, &c);
   if (rc != ISA_OK) return rc;
@@ -626,6 +659,7 @@ size_t isa_dense_workspace_size(int d) {
 
 int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* q, const uint16_t* k,
                        const uint16_t* v, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("isa_dense_attn_fwd");
   if (B < 1 || H < 1 || N < 1 || !std::isfinite(scale)) return ISA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ISA_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(B) * H;

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 namespace isa {
 
@@ -48,6 +49,26 @@ struct FlashParams {
   float* o_part;          // [CTAs, 256, D] fp32 partial accumulators
   float2* ml_part;        // [CTAs, 256] (reference max in log2 units, sum)
   int split_capacity;     // CTAs the partial buffers hold (0 = no split)
+};
+
+// ISA_OK for cudaSuccess; otherwise records e as the calling thread's last
+// CUDA error (isa_last_error) and returns ISA_ERR_CUDA.
+int record_cuda_status(cudaError_t e);
+
+// NVTX ranges around the C entry points, for timelines in a profiler.  Off
+// unless the environment variable ISA_NVTX is set to anything but "0" (read
+// once per process); when off, a range costs one branch.
+bool nvtx_enabled();
+struct NvtxRange {
+  bool on;
+  explicit NvtxRange(const char* name) : on(nvtx_enabled()) {
+    if (on) nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (on) nvtxRangePop();
+  }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
 // Bytes per CTA of key-split partials for head dim D.

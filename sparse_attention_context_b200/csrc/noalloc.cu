@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "isa.h"
+#include "isa_internal.h"
 
 namespace {
 
@@ -26,13 +27,17 @@ void* g_scratch_dev[kMaxDevices] = {};
 // first call per device).  Returns an isa_status.
 int scratch_for_current_device(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ISA_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return isa::record_cuda_status(e);
+  if (dev < 0 || dev >= kMaxDevices) return isa::record_cuda_status(cudaErrorInvalidDevice);
   std::lock_guard<std::mutex> lock(g_setup_mu);
   if (g_scratch_dev[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_isa_static_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return ISA_ERR_CUDA;
+    e = cudaGetSymbolAddress(&p, g_isa_static_scratch);
+    if (e == cudaSuccess && p == nullptr) e = cudaErrorInvalidSymbol;
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // take it out of the runtime's last-error slot; isa_last_error keeps it
+      return isa::record_cuda_status(e);
     }
     g_scratch_dev[dev] = p;
   }
@@ -44,6 +49,7 @@ int scratch_for_current_device(void** out) {
 
 extern "C" int isa_forward_static(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                   uint16_t* out, void* stream) {
+  isa::NvtxRange nvtx_("isa_forward_static");
   const size_t need = isa_workspace_size(shape);
   // invalid or unsupported shape: isa_forward reports which, before any launch
   if (need == 0) return isa_forward(shape, q, k, v, out, nullptr, 0, stream);
@@ -53,6 +59,7 @@ extern "C" int isa_forward_static(const isa_shape* shape, const uint16_t* q, con
   if (rc != ISA_OK) return rc;
   // The control block (device status word, fault-injection word) must start
   // at zero; everything else in the scratch is written before it is read.
-  if (cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ISA_ERR_CUDA;
+  const cudaError_t e = cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return isa::record_cuda_status(e);
   return isa_forward(shape, q, k, v, out, ws, kStaticScratchBytes, stream);
 }

@@ -5,9 +5,10 @@
 // [b*blk, min((b+1)*blk, N_src)), context blocks cover the context rows the
 // same way; the last block of each segment may be partial.  One CTA reduces
 // one block of one (b, h) for all three tensors: 16-byte vector loads (8
-// bf16), fp32 accumulation in a fixed order, a two-level reduction (lane
-// halves by shuffle, row groups through shared memory).  HBM-bound: every
-// byte of q, k, v is read once.
+// bf16), fp32 accumulation in a fixed order: each thread sums one 8-column
+// chunk over a strided set of rows, then the row groups' partial sums are
+// added through shared memory.  HBM-bound: every byte of q, k, v is read
+// once.
 #include "isa_internal.h"
 #include "tc_ptx.cuh"
 

@@ -22,9 +22,12 @@ def shard_heads(H: int, world: int, rank: int) -> tuple[int, int]:
 
 def gather_heads(local, group=None):
     """All-gather of per-rank head slices [B, H_r, N, d] into the whole
-    [B, H, N, d] on every rank, in rank order.  Every rank must hold the
-    same number of heads (H divisible by the world size).  Uses the default
-    process group (or `group`); a single process returns `local` itself."""
+    [B, H, N, d] on every rank, in rank order.  The slices may differ in
+    size by any amount (``shard_heads`` gives the first H % world ranks one
+    head more): each rank pads its slice to the largest H_r, one all-gather
+    moves the padded slices, and every rank keeps the first H_r heads of
+    each.  Uses the default process group (or `group`); a single process
+    returns `local` itself."""
     import torch
     import torch.distributed as dist
 
@@ -35,8 +38,14 @@ def gather_heads(local, group=None):
         return local
     sizes = [torch.zeros(1, dtype=torch.int64, device=local.device) for _ in range(world)]
     dist.all_gather(sizes, torch.tensor([local.shape[1]], dtype=torch.int64, device=local.device), group=group)
-    if len({int(s.item()) for s in sizes}) != 1:
-        raise ValueError("gather_heads needs the same number of heads on every rank")
-    parts = [torch.empty_like(local) for _ in range(world)]
-    dist.all_gather(parts, local.contiguous(), group=group)
-    return torch.cat(parts, dim=1)
+    hs = [int(s.item()) for s in sizes]
+    hmax = max(hs)
+    B, h_r = local.shape[0], local.shape[1]
+    if h_r == hmax:
+        send = local.contiguous()
+    else:
+        send = torch.zeros((B, hmax, *local.shape[2:]), dtype=local.dtype, device=local.device)
+        send[:, :h_r] = local
+    parts = [torch.empty_like(send) for _ in range(world)]
+    dist.all_gather(parts, send, group=group)
+    return torch.cat([p[:, :h] for p, h in zip(parts, hs)], dim=1)

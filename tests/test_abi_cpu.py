@@ -109,3 +109,25 @@ def test_status_strings(L):
     assert L.isa_status_string(0) == b"ok"
     assert b"timed out" in L.isa_status_string(5)
     assert L.isa_status_string(99) == b"unknown status"
+
+
+def test_nvtx_ranges_opt_in():
+    """With ISA_NVTX=1 every entry point opens and closes an NVTX range (a
+    no-op without a profiler attached); argument validation still returns
+    its status.  Run in a fresh process, since the variable is read once."""
+    import subprocess
+    import sys
+
+    code = (
+        "import ctypes\n"
+        "from sparse_attention_context_b200 import _lib\n"
+        "L = _lib.lib()\n"
+        "s = _lib.IsaShape(1, 2, 256, 256, 96, 64, 0.5, 0.25, 0.0)\n"
+        "buf = (ctypes.c_uint8 * 1024)(); p = ctypes.addressof(buf)\n"
+        "assert L.isa_forward(ctypes.byref(s), p, p, p, p, p, 1024, None) == 2\n"
+        "assert L.isa_dense_attn_fwd(1, 1, 0, 64, 0.0, p, p, p, p, p, 256, None) == 1\n"
+        "print('ok')\n")
+    for flag in ("1", "0"):
+        r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=120,
+                           env=dict(os.environ, ISA_NVTX=flag))
+        assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr

@@ -55,3 +55,29 @@ def test_bad_route_index_is_flagged_not_faulted(cuda_ok):
     routed[0, 0, 0] = cfg.N + 5
     api.isa_attn_fwd(q, k, v, kept, routed, taylor, shape, ws)
     assert api.isa_read_device_status(ws) == 1
+
+
+def test_timed_out_key_split_writes_no_rows(cuda_ok):
+    """A full-attention launch whose items run split along the keys: after
+    an (injected) timeout no piece writes partials, so the merge must leave
+    the rows unwritten instead of combining stale partial buffers."""
+    cfg = CONFIGS["tiny"].replace(H=1, d=128, N_src=3000, N_ctx=2900, block=128, keep=0.35, rho=0.25)
+    _, (q, k, v) = inputs(cfg)
+    shape = api.make_shape(q, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    ws = api.new_workspace(shape)
+    out = torch.empty_like(q)
+    kept, _ = api.isa_preselect_ctx(q, k, v, shape, ws)
+    routed, taylor, _ = api.isa_route_queries(q, kept, shape, ws)
+    api.isa_full_attn_fwd(q, k, v, kept, routed, shape, ws, out)  # fills the partial buffers
+    assert api.isa_read_device_status(ws) == 0
+    good = out.clone()
+    sentinel = torch.full_like(q, 7.0)
+    ws[4:8].view(torch.int32).fill_(1)
+    api.isa_full_attn_fwd(q, k, v, kept, routed, shape, ws, sentinel)
+    assert api.isa_read_device_status(ws) == 5
+    assert bool((sentinel == 7.0).all()), "rows written after a timeout"
+    ws[4:8].view(torch.int32).fill_(0)
+    api.isa_full_attn_fwd(q, k, v, kept, routed, shape, ws, sentinel)
+    assert api.isa_read_device_status(ws) == 0
+    r = routed[0, 0].long()
+    assert torch.equal(sentinel[0, 0, r].view(torch.int16), good[0, 0, r].view(torch.int16))

@@ -66,7 +66,7 @@ def test_two_ranks_reduce_timing_and_run_own_replicas(tmp_path):
     assert not np.array_equal(res[0]["q_head"], res[1]["q_head"])  # each replica draws its own inputs
 
 
-def _shard_worker(rank, world, port, out_dir):
+def _shard_worker(rank, world, port, out_dir, H=4):
     import datetime
 
     import torch
@@ -79,7 +79,7 @@ def _shard_worker(rank, world, port, out_dir):
 
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        cfg = CONFIGS["tiny"].replace(H=4, N_src=96, N_ctx=64)
+        cfg = CONFIGS["tiny"].replace(H=H, N_src=96, N_ctx=64)
         h0, h1 = shard_heads(cfg.H, world, rank)
         local = to_torch_bf16(make_inputs(cfg, seed=0, heads=range(h0, h1))[0])
         full = gather_heads(local)  # stands in for the output slices of the per-rank forwards
@@ -89,17 +89,18 @@ def _shard_worker(rank, world, port, out_dir):
         dist.destroy_process_group()
 
 
-def test_head_shards_gather_to_the_whole_problem(tmp_path):
+@pytest.mark.parametrize("H,world", [(4, 2), (7, 3)])
+def test_head_shards_gather_to_the_whole_problem(tmp_path, H, world):
     """Each rank draws only its heads of one seeded problem; the gathered
-    slices equal the whole problem drawn in one process, on every rank."""
+    slices equal the whole problem drawn in one process, on every rank.
+    7 heads over 3 ranks gives slices of 3, 2 and 2 heads."""
     import torch
 
     from workloads import CONFIGS, make_inputs, to_torch_bf16
 
-    world = 2
-    mp.start_processes(_shard_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+    mp.start_processes(_shard_worker, args=(world, _free_port(), str(tmp_path), H), nprocs=world, join=True,
                        start_method="spawn")
-    cfg = CONFIGS["tiny"].replace(H=4, N_src=96, N_ctx=64)
+    cfg = CONFIGS["tiny"].replace(H=H, N_src=96, N_ctx=64)
     whole = to_torch_bf16(make_inputs(cfg, seed=0)[0])
     for r in range(world):
         got = torch.load(tmp_path / f"full{r}.pt")
