@@ -10,6 +10,13 @@
  *                                        -> O2 [128, d] fp32 = P V  (P from tensor memory)
  * d and bn in {64, 128}.  ws: >= 256 bytes, zeroed; its first int32 receives
  * ISA_ERR_DEVICE_TIMEOUT if a bounded wait expires.  Asynchronous on stream.
+ *
+ * isa_selftest_ex2 evaluates the softmax's exponentials on n given fp32
+ * arguments x (device pointers, n >= 0): y_poly = the FMA-pipe 2^x of the
+ * attention kernels (Cody-Waite reduction, minimax cubic; arguments taken in
+ * pairs as the kernels do), y_mufu = the MUFU ex2.approx.ftz used for the
+ * other exponentials, y_ref = CUDA's exp2f.  Asynchronous on stream;
+ * ISA_ERR_INVALID_ARG for n < 0 or a null pointer when n > 0.
  */
 #ifndef ISA_SELFTEST_H_
 #define ISA_SELFTEST_H_
@@ -19,6 +26,7 @@ extern "C" {
 #endif
 int isa_selftest_umma(int d, int bn, const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V,
                       float* S, float* O, float* O2, void* ws, void* stream);
+int isa_selftest_ex2(const float* x, float* y_poly, float* y_mufu, float* y_ref, int n, void* stream);
 #ifdef __cplusplus
 }
 #endif

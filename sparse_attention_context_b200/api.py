@@ -362,3 +362,14 @@ def isa_selftest_umma(A, B, P, V, ws, stream=None):
                                  O.data_ptr(), O2.data_ptr(), ws.data_ptr(), _stream(stream))
     check("isa_selftest_umma", rc)
     return S, O, O2
+
+
+def isa_selftest_ex2(x, stream=None):
+    """Test-only: (FMA-pipe 2^x of the softmax, MUFU ex2, exp2f) of the fp32
+    CUDA tensor x, each a tensor like x."""
+    if not (x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()):
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    yp, ym, yr = (torch.empty_like(x) for _ in range(3))
+    rc = lib().isa_selftest_ex2(x.data_ptr(), yp.data_ptr(), ym.data_ptr(), yr.data_ptr(), x.numel(), _stream(stream))
+    check("isa_selftest_ex2", rc)
+    return yp, ym, yr

@@ -3,8 +3,10 @@
 // threads into the 128B-swizzled layout, B loaded by TMA) and O = P V with
 // V MN-major (loaded by TMA), both accumulated in TMEM and read back with
 // tcgen05.ld; and O2 = P V with P written by threads into TMEM (tcgen05.st,
-// two bf16 per column) and read by the UMMA as its A operand.  Exported for
-// the tests only (include/isa_selftest.h).
+// two bf16 per column) and read by the UMMA as its A operand.  Also the
+// exponentials of the softmax: the FMA-pipe 2^x (ex2_poly2) and the MUFU
+// ex2 on given arguments, beside CUDA's exp2f.  Exported for the tests
+// only (include/isa_selftest.h).
 #include "isa.h"
 #include "isa_internal.h"
 #include "isa_selftest.h"
@@ -156,7 +158,37 @@ static int run_probe(const uint16_t* A, const uint16_t* B, const uint16_t* P, co
   return cudaGetLastError() == cudaSuccess ? ISA_OK : ISA_ERR_CUDA;
 }
 
+// y_poly = ex2_poly2(x) (two arguments per call, as the softmax uses it),
+// y_mufu = ex2.approx.ftz (the MUFU path), y_ref = exp2f; one thread per pair.
+__global__ void __launch_bounds__(256) ex2_probe_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                                                        float* __restrict__ y_mufu, float* __restrict__ y_ref,
+                                                        int n) {
+  const int i = 2 * (blockIdx.x * 256 + threadIdx.x);
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  const float2 a = make_float2(x[i], two ? x[i + 1] : 0.f);
+  const float2 e = ex2_poly2(a);
+  y_poly[i] = e.x;
+  y_mufu[i] = ex2(a.x);
+  y_ref[i] = exp2f(a.x);
+  if (two) {
+    y_poly[i + 1] = e.y;
+    y_mufu[i + 1] = ex2(a.y);
+    y_ref[i + 1] = exp2f(a.y);
+  }
+}
+
 }  // namespace isa
+
+extern "C" int isa_selftest_ex2(const float* x, float* y_poly, float* y_mufu, float* y_ref, int n, void* stream) {
+  if (n < 0) return ISA_ERR_INVALID_ARG;
+  if (n == 0) return ISA_OK;
+  if (!x || !y_poly || !y_mufu || !y_ref) return ISA_ERR_INVALID_ARG;
+  const int pairs = (n + 1) / 2;
+  isa::ex2_probe_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_mufu,
+                                                                                            y_ref, n);
+  return isa::record_cuda_status(cudaGetLastError());
+}
 
 extern "C" int isa_selftest_umma(int d, int bn, const uint16_t* A, const uint16_t* B, const uint16_t* P,
                                  const uint16_t* V, float* S, float* O, float* O2, void* ws, void* stream) {

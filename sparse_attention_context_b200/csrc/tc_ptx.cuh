@@ -288,21 +288,23 @@ __device__ __forceinline__ float ex2(float x) {
 // 2^x for two values on the FMA pipe, packed fp32x2 (relieves the MUFU
 // pipe, which the exponentials of a softmax otherwise saturate).  Method:
 // Cody-Waite range reduction x = n + f, n = rint(x) by the 1.5*2^23
-// round-to-integer addition, f in [-0.5, 0.5]; 2^f by a cubic with
-// coefficients from a Remez exchange for minimal relative error on that
-// interval (max relative error 7.5e-5, 1.5e-4 in fp32 arithmetic, below
-// the 2^-9 of the bf16 rounding that follows); 2^n applied by
-// adding n to the exponent field.  x is clamped at -126 so that the result
-// stays a normal float (2^-126 is far below anything a softmax keeps).
+// round-to-integer addition, f in [-0.5, 0.5]; 2^f by the cubic of least
+// maximum relative error on that interval, found by a Remez exchange
+// (tests/golden/ex2_cubic_fit.py prints these coefficients; max relative
+// error 7.5e-5, about 1.5e-4 in fp32 arithmetic, below the 2^-9 of the bf16
+// rounding that follows); 2^n applied by adding n to the exponent field.
+// x is clamped at -126: results are normal floats down to 2^-125.5 and at
+// most 1e-4 of 2^-126 below it at the clamp (far below anything a softmax
+// keeps).  Valid for x up to 127 (the softmax passes x <= 32).
 __device__ __forceinline__ float2 ex2_poly2(float2 x) {
   x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
   const float2 M = make_float2(12582912.f, 12582912.f);
   const float2 t = __fadd2_rn(x, M);                                     // n in t's low mantissa bits
   const float2 f = __fadd2_rn(x, __fadd2_rn(M, make_float2(-t.x, -t.y)));  // x - n
-  float2 q = __ffma2_rn(make_float2(0.05517166853f, 0.05517166853f), f,
-                        make_float2(0.24261112511f, 0.24261112511f));
-  q = __ffma2_rn(q, f, make_float2(0.69326096773f, 0.69326096773f));
-  q = __ffma2_rn(q, f, make_float2(0.99992805719f, 0.99992805719f));
+  float2 q = __ffma2_rn(make_float2(0.05517166906f, 0.05517166906f), f,
+                        make_float2(0.24261112219f, 0.24261112219f));
+  q = __ffma2_rn(q, f, make_float2(0.69326098546f, 0.69326098546f));
+  q = __ffma2_rn(q, f, make_float2(0.99992807354f, 0.99992807354f));
   return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }

@@ -115,8 +115,6 @@ def compare_head(cfg: Config, bits, g, b, h, keep, rho, rows=None):
     if not same_routed:
         ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, keep, rho, kept_override=kept_gpu,
                               routed_override=routed_gpu, rows=rows)
-    elif rows is not None:
-        ref = oracle.isa_head(q, k, v, cfg.N_src, cfg.block, keep, rho, kept_override=kept_gpu, rows=rows)
     # stages 3 + 4
     o_gpu = g["out"][b, h]
     sel = slice(None) if rows is None else rows

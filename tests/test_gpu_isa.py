@@ -61,24 +61,27 @@ def test_keep1_rho1_equals_dense_kernel_path(cuda_ok):
     check_out(out.double().cpu().numpy(), dense.double().cpu().numpy(), "isa vs dense")
 
 
-@pytest.mark.parametrize("name,heads", [("480p", None), ("720p", [0, 39])])
+@pytest.mark.parametrize("name,heads", [("480p", None), ("720p", [0, 5, 11, 16, 22, 27, 33, 39])])
 def test_isa_full_size_sampled(cuda_ok, name, heads):
     """Full-size DiT latents through the fused path that isa_forward and the
     bench run.  480p runs all 24 heads in the launch configuration the bench
-    times; 720p runs two of its 40 heads (heads are independent units).
-    Sets are checked whole, outputs on sampled rows."""
+    times and checks every head; 720p runs 8 of its 40 heads (heads are
+    independent units).  Per head the saliency, kept set, sharpness and
+    routed / Taylor sets are checked whole against the oracle, the outputs
+    on sampled rows of both paths plus the segment edges."""
     cfg = CONFIGS[name]
     bits, (q, k, v) = inputs(cfg, heads=heads)
     H = q.shape[1]
     g = run_fused(cfg.replace(H=H), q, k, v)
     assert g["status"] == 0
     rng = np.random.default_rng(7)
-    for h in sorted({0, H - 1}):
+    per_head = 48 if H > 8 else 96
+    for h in range(H):
         nr = g["routed"].shape[-1]
         routed = g["routed"][0, h]
         taylor = g["taylor"][0, h]
         rows = np.unique(np.concatenate([
-            rng.choice(routed, min(96, nr), replace=False), rng.choice(taylor, 96, replace=False),
+            rng.choice(routed, min(per_head, nr), replace=False), rng.choice(taylor, per_head, replace=False),
             [0, cfg.N_src - 1, cfg.N_src, cfg.N - 1]]))
         compare_head(cfg.replace(H=H), bits, g, 0, h, cfg.keep, cfg.rho, rows=rows)
 
