@@ -713,25 +713,31 @@ def main():
         assert api.isa_read_device_status(dws) == 0
         del dout
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: the C entry point
+    # isa_forward_host (copies in, forward, copy out, pipelined over head
+    # slices), every step a whole call that returns once the output is in
+    # pinned host memory
     e2e = None
     if not args.no_e2e:
         hq, hk, hv = (to_torch_bf16(b).pin_memory() for b in bits)
         hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        staging = torch.empty(api.host_staging_size(shape), dtype=torch.uint8, device=dev)
         for _ in range(2):
-            api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws, out=hout)
+            api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, out=hout, staging=staging)
         barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ne = max(2, min(args.steps, 5))
+        ne = args.steps
         e0.record(stream)
         for _ in range(ne):
-            api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, ws=ws, out=hout)
+            api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, out=hout, staging=staging)
         e1.record(stream)
         torch.cuda.synchronize()
+        assert api.isa_read_device_status(staging) == 0
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / ne, dev)
         e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": 3 * q.numel() * 2,
-               "d2h_bytes_per_step": q.numel() * 2}
+               "d2h_bytes_per_step": q.numel() * 2, "steps": ne,
+               "path": "isa_forward_host (C ABI), pinned host buffers, default head slices"}
 
     gather_ms = None
     if args.shard == "heads" and args.gather and world > 1:

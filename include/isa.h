@@ -243,6 +243,40 @@ int isa_forward(const isa_shape* shape, const uint16_t* q, const uint16_t* k, co
 int isa_forward_static(const isa_shape* shape, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                        uint16_t* out, void* stream);
 
+/* All four stages on HOST buffers, end to end: copies q, k, v in, runs the
+ * forward and copies out back, for callers whose tensors live in host
+ * memory.  (The ISA pages have no counterpart; this is a packaging of the
+ * same path.)  Every (b, h) is independent, so the B*H heads are taken in
+ * `groups` consecutive slices (groups <= 0: two heads a slice from 8 heads
+ * on, else one slice); the copy-in of a slice on stream_in, the forward of
+ * the one before on stream_compute (isa_forward on the slice) and the
+ * copy-out of the one before that on stream_out run at once, so both PCIe
+ * directions overlap the kernels.  Each (b, h) gets the same index sets as
+ * under isa_forward; only the merge of the full-attention key-split tail
+ * can round differently (it depends on how many heads share a launch).
+ *   hq, hk, hv   [B, H, N, d] bf16 in (pinned host memory for asynchronous
+ *                copies; pageable memory works, with synchronous copies).
+ *   hout         [B, H, N, d] bf16 out (host memory).
+ *   staging      device buffer of staging_bytes >= isa_host_staging_size(
+ *                shape, groups) bytes, 16-byte aligned, owned by the caller:
+ *                a workspace for one slice (its first 256 bytes are the
+ *                control block; isa_read_device_status(staging, ...) reads
+ *                its status word) and a ring of up to 3 slices of q, k, v,
+ *                out.  Nothing else is allocated on the device.
+ *   streams      stream_in / stream_out may be NULL (then stream_compute is
+ *                used for the copies too, without overlap).
+ * The call returns once everything is enqueued; the last copy-out is
+ * ordered before any later work on stream_compute, so synchronising
+ * stream_compute makes hout complete.  hq, hk, hv must not change and hout
+ * must not be read before then.  Argument errors return before anything is
+ * enqueued; an error from a slice's isa_forward is returned as it is, with
+ * earlier slices already enqueued.  isa_host_staging_size returns 0 for an
+ * invalid shape. */
+size_t isa_host_staging_size(const isa_shape* shape, int groups);
+int isa_forward_host(const isa_shape* shape, const uint16_t* hq, const uint16_t* hk, const uint16_t* hv,
+                     uint16_t* hout, void* staging, size_t staging_bytes, int groups, void* stream_compute,
+                     void* stream_in, void* stream_out);
+
 /* In-house dense flash attention (the latency baseline; equals ISA at
  * keep = rho = 1): out = softmax(scale q k^T) v over all N keys, per (b, h),
  * non-causal.  scale <= 0 selects 1/sqrt(d).  ws: a zeroed buffer of

@@ -54,6 +54,8 @@ SIGNATURES = {
     "isa_forward_taylor1": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P, _SZ, _P]),
     "isa_forward": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_forward_static": (_I, [_SH, _P, _P, _P, _P, _P]),
+    "isa_host_staging_size": (_SZ, [_SH, _I]),
+    "isa_forward_host": (_I, [_SH, _P, _P, _P, _P, _P, _SZ, _I, _P, _P, _P]),
     "isa_dense_workspace_size": (_SZ, [_I]),
     "isa_dense_attn_fwd": (_I, [_I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P]),
     "isa_read_device_status": (_I, [_P, _P]),

@@ -227,18 +227,19 @@ def isa_forward_taylor1(q, k, v, N_src: int, block: int, keep: float, rho: float
 
 
 def isa_forward(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, ws=None, out=None,
-                stream=None, groups=None):
+                stream=None, groups=None, staging=None, sync=True):
     """All ISA stages in one call.
 
-    CUDA inputs: runs on the current stream and returns a CUDA tensor.
-    CPU inputs (the host-buffer path): copies q, k, v to the GPU, runs, and
-    copies the output back into a pinned CPU tensor (returned).  Every
-    (b, h) is an independent unit, so the heads are taken in `groups`
-    consecutive slices (default: two heads a slice from 8 heads on): the
-    host-to-device copy of a slice, the forward of the previous slice and the
-    device-to-host copy of the one before run on three streams at once, and
-    PCIe transfers in both directions overlap the GPU work.  Pass pinned
-    host tensors for the copies to be asynchronous.
+    CUDA inputs: isa_forward on the current stream; returns a CUDA tensor.
+    CPU inputs (the host-buffer path): isa_forward_host, which copies q, k, v
+    in, runs the forward and copies the output back into a (pinned) CPU
+    tensor, head slices pipelined over a copy-in stream, the current stream
+    and a copy-out stream (`groups` slices; None lets the library choose).
+    `staging` is the device buffer the library works in (allocated here when
+    None or too small).  With sync=True (default) the call returns once the
+    output is in host memory; with sync=False it returns at once and the
+    output is complete when the current stream is.  Pass pinned host tensors
+    for the copies to be asynchronous.
     """
     if q.is_cuda:
         shape = make_shape(q, N_src, block, keep, rho, scale)
@@ -250,64 +251,51 @@ def isa_forward(q, k, v, N_src: int, block: int, keep: float, rho: float, scale:
                                ws.data_ptr(), ws.numel(), _stream(stream))
         check("isa_forward", rc)
         return o
-    return _isa_forward_host(q, k, v, N_src, block, keep, rho, scale, ws, out, groups)
+    return isa_forward_host(q, k, v, N_src, block, keep, rho, scale, out=out, groups=groups, staging=staging,
+                            stream=stream, sync=sync)
 
 
-def _isa_forward_host(q, k, v, N_src, block, keep, rho, scale, ws, out, groups):
-    """Host-buffer path of isa_forward: head slices pipelined over a copy-in
-    stream, the caller's current stream (compute) and a copy-out stream."""
-    dev = torch.device("cuda")
-    B, H, N, d = q.shape
-    BH = B * H
-    G = groups if groups is not None else (BH // 2 if BH >= 8 else 1)  # two heads a slice (measured best at 480p)
-    G = max(1, min(int(G), BH))
-    bounds = [BH * i // G for i in range(G + 1)]
-    qf, kf, vf = (t.reshape(BH, N, d) for t in (q, k, v))
-    dq, dk, dv = (torch.empty((BH, N, d), dtype=q.dtype, device=dev) for _ in range(3))
-    do = torch.empty((BH, N, d), dtype=q.dtype, device=dev)
-    dst = out if out is not None else torch.empty((B, H, N, d), dtype=q.dtype, pin_memory=True)
-    dstf = dst.reshape(BH, N, d)
-    comp = torch.cuda.current_stream()
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    start = torch.cuda.Event()
-    start.record(comp)
-    s_in.wait_event(start)
-    s_out.wait_event(start)
-    big = max(bounds[i + 1] - bounds[i] for i in range(G))
-    shape_big = make_shape(torch.empty((1, big, N, d), device="meta"), N_src, block, keep, rho, scale)
-    if ws is None or ws.numel() < lib().isa_workspace_size(ctypes.byref(shape_big)):
-        ws = new_workspace(shape_big, dev)
-    done_in, done_comp = [], []
-    for g in range(G):
-        a, b = bounds[g], bounds[g + 1]
-        with torch.cuda.stream(s_in):
-            for src, buf in ((qf, dq), (kf, dk), (vf, dv)):
-                buf[a:b].copy_(src[a:b], non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(s_in)
-            done_in.append(ev)
-    for g in range(G):
-        a, b = bounds[g], bounds[g + 1]
-        comp.wait_event(done_in[g])
-        shape = make_shape(torch.empty((1, b - a, N, d), device="meta"), N_src, block, keep, rho, scale)
-        rc = lib().isa_forward(ctypes.byref(shape), dq[a].data_ptr(), dk[a].data_ptr(), dv[a].data_ptr(),
-                               do[a].data_ptr(), ws.data_ptr(), ws.numel(), _stream(None))
-        check("isa_forward", rc)
-        ev = torch.cuda.Event()
-        ev.record(comp)
-        done_comp.append(ev)
-    with torch.cuda.stream(s_out):
-        for g in range(G):
-            a, b = bounds[g], bounds[g + 1]
-            s_out.wait_event(done_comp[g])
-            dstf[a:b].copy_(do[a:b], non_blocking=True)
-    fin = torch.cuda.Event()
-    fin.record(s_out)
-    comp.wait_event(fin)
-    comp.synchronize()
-    for t in (dq, dk, dv, do, ws):  # keep the caching allocator from reusing them early
-        t.record_stream(s_in)
-        t.record_stream(s_out)
+_COPY_STREAMS = {}
+
+
+def _copy_streams(device):
+    """One copy-in and one copy-out stream per device, made once."""
+    key = torch.device(device).index
+    if key not in _COPY_STREAMS:
+        with torch.cuda.device(key):
+            _COPY_STREAMS[key] = (torch.cuda.Stream(), torch.cuda.Stream())
+    return _COPY_STREAMS[key]
+
+
+def host_staging_size(shape: IsaShape, groups=None) -> int:
+    return lib().isa_host_staging_size(ctypes.byref(shape), 0 if groups is None else int(groups))
+
+
+def isa_forward_host(q, k, v, N_src: int, block: int, keep: float, rho: float, scale: float = 0.0, out=None,
+                     groups=None, staging=None, stream=None, sync=True):
+    """The C entry point isa_forward_host on CPU bf16 tensors [B, H, N, d].
+    Returns the output as a CPU tensor (pinned unless `out` is given)."""
+    for t in (q, k, v) + ((out,) if out is not None else ()):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("host path: q, k, v, out must be contiguous CPU bf16 tensors [B, H, N, d]")
+    shape = make_shape(q, N_src, block, keep, rho, scale)
+    G = 0 if groups is None else int(groups)
+    n = lib().isa_host_staging_size(ctypes.byref(shape), G)
+    if n == 0:
+        raise ValueError("invalid or unsupported shape")
+    comp = torch.cuda.current_stream() if stream is None else stream
+    dev = comp.device
+    if staging is None or staging.numel() < n:
+        staging = torch.empty(n, dtype=torch.uint8, device=dev)
+    dst = out if out is not None else torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    s_in, s_out = _copy_streams(dev)
+    rc = lib().isa_forward_host(ctypes.byref(shape), q.data_ptr(), k.data_ptr(), v.data_ptr(), dst.data_ptr(),
+                                staging.data_ptr(), staging.numel(), G, comp.cuda_stream, s_in.cuda_stream,
+                                s_out.cuda_stream)
+    check("isa_forward_host", rc)
+    staging.record_stream(comp)  # the caching allocator keeps it until the enqueued work is done
+    if sync:
+        comp.synchronize()
     return dst
 
 

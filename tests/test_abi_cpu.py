@@ -131,3 +131,29 @@ def test_nvtx_ranges_opt_in():
         r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=120,
                            env=dict(os.environ, ISA_NVTX=flag))
         assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+
+
+def test_host_staging_size_and_validation(L):
+    """isa_host_staging_size: a slice workspace plus a ring of up to three
+    slices of q, k, v, out; isa_forward_host rejects bad arguments before
+    enqueuing anything."""
+    s = shape()  # 480p: 24 heads
+    ws2 = L.isa_workspace_size(ctypes.byref(shape(H=2)))
+    head = 40560 * 128 * 2
+    n_default = L.isa_host_staging_size(ctypes.byref(s), 0)   # 12 slices of 2 heads
+    assert n_default >= ws2 + 3 * 4 * 2 * head
+    assert n_default < ws2 + 3 * 4 * 2 * head + 64 * 1024
+    n1 = L.isa_host_staging_size(ctypes.byref(s), 1)          # one slice of all 24 heads
+    assert n1 >= L.isa_workspace_size(ctypes.byref(s)) + 4 * 24 * head
+    assert L.isa_host_staging_size(ctypes.byref(s), 100) == L.isa_host_staging_size(ctypes.byref(s), 24)
+    assert L.isa_host_staging_size(ctypes.byref(shape(d=96)), 0) == 0
+    buf = (ctypes.c_uint8 * 4096)()
+    p = (ctypes.addressof(buf) + 255) // 256 * 256
+    t = shape(H=2, N_src=256, N_ctx=256, d=64, block=64)
+    need = L.isa_host_staging_size(ctypes.byref(t), 0)
+    assert L.isa_forward_host(ctypes.byref(shape(d=96)), p, p, p, p, p, need, 0, None, None, None) == 2
+    assert L.isa_forward_host(ctypes.byref(shape(keep=2.0)), p, p, p, p, p, need, 0, None, None, None) == 1
+    assert L.isa_forward_host(ctypes.byref(t), None, p, p, p, p, need, 0, None, None, None) == 1
+    assert L.isa_forward_host(ctypes.byref(t), p, p, p, None, p, need, 0, None, None, None) == 1
+    assert L.isa_forward_host(ctypes.byref(t), p, p, p, p, p + 8, need, 0, None, None, None) == 1
+    assert L.isa_forward_host(ctypes.byref(t), p, p, p, p, p, need - 1, 0, None, None, None) == 3

@@ -86,19 +86,44 @@ def test_isa_full_size_sampled(cuda_ok, name, heads):
         compare_head(cfg.replace(H=H), bits, g, 0, h, cfg.keep, cfg.rho, rows=rows)
 
 
-@pytest.mark.parametrize("groups", [1, 5, None])
+@pytest.mark.parametrize("groups", [1, 2, 5, None])
 def test_host_buffer_path(cuda_ok, groups):
-    """isa_forward on pinned host tensors (the end-to-end path: head slices
-    pipelined over copy-in, compute and copy-out streams) gives the device
-    path's output: index sets are per head, so only the key-split merge of
-    the full-attention tail (which depends on how many heads share a launch)
-    may round differently."""
+    """isa_forward_host (the end-to-end path: head slices pipelined over
+    copy-in, compute and copy-out streams through a staging ring) gives the
+    device path's output: index sets are per head, so only the key-split
+    merge of the full-attention tail (which depends on how many heads share
+    a launch) may round differently.  Two calls in a row reuse the staging
+    buffer."""
     cfg = CONFIGS["small"]
     bits, (q, k, v) = inputs(cfg)
     ref = api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-    got = api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, groups=groups)
-    assert not got.is_cuda and got.shape == q.shape
-    check_out(got.double().numpy(), ref.double().cpu().numpy(), f"host path, groups={groups}")
-    if groups == 1:
-        assert torch.equal(got.view(torch.int16), ref.cpu().view(torch.int16))  # same launches: same bits
+    shape = api.make_shape(hq, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    staging = torch.zeros(api.host_staging_size(shape, groups), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        got = api.isa_forward(hq, hk, hv, cfg.N_src, cfg.block, cfg.keep, cfg.rho, groups=groups, staging=staging)
+        assert not got.is_cuda and got.shape == q.shape
+        assert api.isa_read_device_status(staging) == 0
+        check_out(got.double().numpy(), ref.double().cpu().numpy(), f"host path, groups={groups}")
+        if groups == 1:
+            assert torch.equal(got.view(torch.int16), ref.cpu().view(torch.int16))  # same launches: same bits
+
+
+def test_host_buffer_path_pageable_and_batch(cuda_ok):
+    """Pageable host memory (synchronous copies) and B > 1 (slices cut
+    across the batch dimension): each head's output as on the device path."""
+    cfg = CONFIGS["tiny"].replace(B=2, H=5, d=128, N_src=700, N_ctx=450, block=128, keep=0.5, rho=0.2)
+    bits, (q, k, v) = inputs(cfg)
+    ref = api.isa_forward(q, k, v, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    got = api.isa_forward(q.cpu(), k.cpu(), v.cpu(), cfg.N_src, cfg.block, cfg.keep, cfg.rho, groups=3)
+    check_out(got.double().numpy(), ref.double().cpu().numpy(), "pageable host path")
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            compare_head(cfg, bits, dict(out=got.double().numpy(), **_sets(q, k, v, cfg)), b, h, cfg.keep, cfg.rho)
+
+
+def _sets(q, k, v, cfg):
+    """Index sets and statistics of the device path (per head they are what
+    the host path computes too)."""
+    g = run_fused(cfg, q, k, v)
+    return {key: g[key] for key in ("kept", "sal", "sharp", "routed", "taylor")}
