@@ -171,25 +171,6 @@ __global__ void __launch_bounds__(352, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  // The last key tile of an item runs its QK^T only over the columns that
-  // hold kept blocks (rounded up to 16); the softmax still reads all 128 S
-  // columns and masks the rest with the -inf key bias, which needs finite
-  // values there: zero them once (later tiles leave finite scores behind).
-  if (warp < 8) {
-    const uint32_t z_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint32_t z[32];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) z[c] = 0u;
-#pragma unroll
-    for (int j = 0; j < BN / 32; ++j) tmem_st32(tmem + z_lane + (warp >> 2) * BN + j * 32, z);
-    tmem_wait_st();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // valid key columns of an item's last key tile, rounded up to the UMMA's
-  // N granularity of 16 (nK = nSB + n_keep kept blocks, nT tiles of 128)
-  const int n_last = ((p.nSB + p.n_keep - (nT - 1) * BN) + 15) & ~15;
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -233,7 +214,6 @@ __global__ void __launch_bounds__(352, 1)
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       constexpr uint32_t IDS = idesc_bf16(128, BN, 0);
-      const uint32_t IDS_last = idesc_bf16(128, n_last, 0);
       constexpr uint32_t IDO = idesc_bf16(128, D, 1);
       bool ok = true;
       // S_i(g) = Q_i (hi + lo) of key tile g, chunk by chunk of K: S_0 waits
@@ -243,7 +223,6 @@ __global__ void __launch_bounds__(352, 1)
         const int k = g / nT;
         const uint32_t qa = aQ + ((k & 1) * 2 + i) * C::Q_BYTES;
         const uint32_t dS = tmem + i * BN;
-        const uint32_t ids = (g % nT == nT - 1) ? IDS_last : IDS;  // last tile: only its kept columns
 #pragma unroll
         for (int cc = 0; cc < C::NKC; ++cc) {
           const int c = cc % (D / 64);
@@ -254,7 +233,7 @@ __global__ void __launch_bounds__(352, 1)
           }
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4)
-            umma_bf16(dS, desc_k_sw128(qa + c * (128 * 128) + k4 * 32), desc_k_sw128(kb + k4 * 32), ids,
+            umma_bf16(dS, desc_k_sw128(qa + c * (128 * 128) + k4 * 32), desc_k_sw128(kb + k4 * 32), IDS,
                       (cc > 0 || k4 > 0) ? 1u : 0u);
           if (i == 1) umma_commit(&bars->k_empty[cc]);
         }
@@ -273,12 +252,10 @@ __global__ void __launch_bounds__(352, 1)
         if (t == 0 && k > 0 && !fw1(&bars->o_free[i], (k - 1) & 1, bars, p)) return false;
         if (!fw1(&bars->p_full[i], g & 1, bars, p)) return false;
         tc_fence_after();
-        const int nkk = (t == nT - 1 ? n_last : BN) / 16;  // k-steps over the tile's computed keys
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          if (kk < nkk)
-            umma_bf16_tmem_a(tmem + 2 * BN + i * D, tmem + i * BN + kk * 8,
-                             desc_mn_sw128(aV + kk * 16 * 128, BN * 128), IDO, (t > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem + 2 * BN + i * D, tmem + i * BN + kk * 8, desc_mn_sw128(aV + kk * 16 * 128, BN * 128),
+                           IDO, (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bars->o_done[i]);
         return true;
       };
@@ -403,11 +380,8 @@ __global__ void __launch_bounds__(352, 1)
         const float mref = (m == -INFINITY) ? 0.f : m;
         const float2 nm2 = make_float2(-mref, -mref);
         float2 ps2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        // quarters holding computed keys (the last tile's PV reads only those)
-        const int nq = t == nT - 1 ? (n_last + 31) / 32 : BN / 32;
 #pragma unroll
         for (int j = 0; j < BN / 32; ++j) {
-          if (j >= nq) break;
           // quarter j: P to columns [16j, 16j + 16) (their scores are in registers)
           const float2* bp = reinterpret_cast<const float2*>(bias + j * 32);
           uint32_t w[16];

@@ -198,32 +198,31 @@ constexpr int kRouteCT = 512;       // threads per CTA
 constexpr int kRouteNW = kRouteCT / 32;
 constexpr int kRouteChunkCap = (200 * 1024) / 4 - 2048;  // keys per CTA held in shared memory
 
-// Exclusive prefix sum of v over the kRouteCT threads in thread order;
-// `total` receives the CTA-wide sum.  ws: >= 32 ints of shared memory.
-__device__ __forceinline__ int block_exclusive_sum_512(int v, int* ws, int& total) {
+// Exclusive prefix sum of v over the kRouteCT threads in thread order, on
+// 64-bit values (two 32-bit counts packed, low + high, which never carry);
+// `total` receives the CTA-wide sum.  ws: >= kRouteNW words of shared
+// memory, free for reuse when this returns.
+__device__ __forceinline__ unsigned long long block_exclusive_sum_512(unsigned long long v, unsigned long long* ws,
+                                                                      unsigned long long& total) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  int incl = v;
+  unsigned long long incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    const unsigned long long n = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += n;
   }
   if (lane == 31) ws[w] = incl;
   __syncthreads();
-  if (w == 0) {
-    int t = lane < kRouteNW ? ws[lane] : 0;
+  unsigned long long before = 0ull, all = 0ull;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += n;
-    }
-    if (lane < kRouteNW) ws[lane] = t;  // inclusive over warps
+  for (int ww = 0; ww < kRouteNW; ++ww) {  // every thread sums the warp totals (16 words, broadcast reads)
+    const unsigned long long t = ws[ww];
+    before += ww < w ? t : 0ull;
+    all += t;
   }
-  __syncthreads();
-  const int off = w ? ws[w - 1] : 0;
-  total = ws[kRouteNW - 1];
+  total = all;
   __syncthreads();  // ws may be reused right after
-  return off + incl - v;
+  return before + incl - v;
 }
 
 __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT)
@@ -238,19 +237,27 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
   const int n = max(0, min(N, c0 + chunk) - c0);  // keys of this CTA: [c0, c0 + n)
   const int trips = (chunk + kRouteCT - 1) / kRouteCT;
   extern __shared__ unsigned rkeys[];                        // [chunk]
-  int* ceq = reinterpret_cast<int*>(rkeys + chunk);          // [trips][NW] equal-to-T keys, then offsets
-  int* csel = ceq + trips * kRouteNW;                        // [trips][NW] routed keys, then offsets
+  int* cgt = reinterpret_cast<int*>(rkeys + chunk);          // [trips][NW] keys > T, then their offsets
+  int* ceq = cgt + trips * kRouteNW;                         // [trips][NW] keys == T, then their offsets
   __shared__ int whist[kRouteNW][257];                       // per warp, padded
   __shared__ int hist[2][256];                               // this chunk's histogram, by pass parity
   __shared__ int cnt2[2];                                    // keys > T, keys == T of this chunk
-  __shared__ unsigned sh_sel;
-  __shared__ int sh_rem;
+  __shared__ unsigned sh_sel[2];                             // each pass's decision, by pass parity
+  __shared__ int sh_rem[2];
   __shared__ int sh_off[2];                                  // routed keys before this chunk, equal keys it takes
-  __shared__ int scan_ws[32];
+  __shared__ unsigned long long scan_ws[kRouteNW];
   const unsigned* u = reinterpret_cast<const unsigned*>(sharp + static_cast<size_t>(bh) * N);
   for (int i = tid; i < n; i += kRouteCT) rkeys[i] = __ldg(u + c0 + i);
+  for (int e = tid; e < kRouteNW * 257; e += kRouteCT) (&whist[0][0])[e] = 0;
   __syncthreads();
 
+  // Radix select, 4 passes of 8 bits.  Per pass: the warps' histograms
+  // (barrier), their sum into this chunk's histogram by 256 threads, which
+  // also clear them for the next pass (cluster barrier: every chunk's
+  // histogram is complete, and every read of the buffer two passes back is
+  // done), warp 0's decision over the 8 chunks (barrier).  The decision
+  // words are double-buffered, so no barrier separates their reads from
+  // the next pass's writes.
   unsigned T = 0u;
   int need_eq = 0;
   const bool partial = n_route > 0 && n_route < N;  // uniform over the cluster
@@ -259,8 +266,6 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
     int remaining = n_route;
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass, buf = pass & 1;
-      for (int e = tid; e < kRouteNW * 257; e += kRouteCT) (&whist[0][0])[e] = 0;
-      __syncthreads();
       for (int i = tid; i < n; i += kRouteCT) {
         const unsigned x = rkeys[i];
         if ((x & pmask) == prefix) atomicAdd(&whist[w][(x >> shift) & 255u], 1);
@@ -269,11 +274,12 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
       if (tid < 256) {
         int t = 0;
 #pragma unroll
-        for (int ww = 0; ww < kRouteNW; ++ww) t += whist[ww][tid];
+        for (int ww = 0; ww < kRouteNW; ++ww) {
+          t += whist[ww][tid];
+          whist[ww][tid] = 0;
+        }
         hist[buf][tid] = t;
       }
-      // every chunk's histogram of this pass is complete (and every read of
-      // the other buffer, two passes back, is done)
       cl.sync();
       if (w == 0) {
         // lane l owns bins 255-8l .. 248-8l (descending): the cluster-wide
@@ -301,8 +307,8 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             if (cum + tot[k] >= remaining) {
-              sh_sel = static_cast<unsigned>(255 - 8 * lane - k);
-              sh_rem = remaining - cum;
+              sh_sel[buf] = static_cast<unsigned>(255 - 8 * lane - k);
+              sh_rem[buf] = remaining - cum;
               break;
             }
             cum += tot[k];
@@ -310,54 +316,56 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
         }
       }
       __syncthreads();
-      prefix |= sh_sel << shift;
+      prefix |= sh_sel[buf] << shift;
       pmask |= 255u << shift;
-      remaining = sh_rem;
-      __syncthreads();
+      remaining = sh_rem[buf];
     }
     T = prefix;
     need_eq = remaining;
   }
 
-  // per (trip, warp): keys equal to T (for their rank among equal keys) and
-  // keys above T; the chunk's totals go to the cluster
-  int gt = 0;
+  // Ordered compaction.  Per (trip, warp): keys above T and keys equal to
+  // T; one exclusive scan of both (packed) in (trip, warp) order gives
+  // every key its counts of greater and of equal keys before it in the
+  // chunk.  Equal keys are routed in index order up to need_eq over the
+  // head, so a key's routed keys before it in the chunk are
+  // gt_before + min(eq_before, take_eq).
   for (int j = 0; j < trips; ++j) {
     const int i = j * kRouteCT + tid;
     const unsigned x = i < n ? rkeys[i] : 0u;
-    const unsigned beq = __ballot_sync(0xffffffffu, partial && i < n && x == T);
     const unsigned bgt = __ballot_sync(0xffffffffu, partial && i < n && x > T);
+    const unsigned beq = __ballot_sync(0xffffffffu, partial && i < n && x == T);
     if (lane == 0) {
+      cgt[j * kRouteNW + w] = __popc(bgt);
       ceq[j * kRouteNW + w] = __popc(beq);
-      gt += __popc(bgt);
     }
   }
   __syncthreads();
   {
-    const int per = (trips * kRouteNW + kRouteCT - 1) / kRouteCT;
-    int loc = 0;
+    const int ne = trips * kRouteNW;
+    const int per = (ne + kRouteCT - 1) / kRouteCT;
+    unsigned long long loc = 0ull;
     for (int k = 0; k < per; ++k) {
       const int e = tid * per + k;
-      if (e < trips * kRouteNW) loc += ceq[e];
+      if (e < ne) loc += static_cast<unsigned long long>(cgt[e]) | (static_cast<unsigned long long>(ceq[e]) << 32);
     }
-    int n_eq;
-    int run = block_exclusive_sum_512(loc, scan_ws, n_eq);
+    unsigned long long total;
+    unsigned long long run = block_exclusive_sum_512(loc, scan_ws, total);
     for (int k = 0; k < per; ++k) {
       const int e = tid * per + k;
-      if (e < trips * kRouteNW) {
-        const int c = ceq[e];
-        ceq[e] = run;
-        run += c;
+      if (e < ne) {
+        const int g = cgt[e], q = ceq[e];
+        cgt[e] = static_cast<int>(run & 0xffffffffull);
+        ceq[e] = static_cast<int>(run >> 32);
+        run += static_cast<unsigned long long>(g) | (static_cast<unsigned long long>(q) << 32);
       }
     }
-    int n_gt;
-    block_exclusive_sum_512(gt, scan_ws, n_gt);
     if (tid == 0) {
-      cnt2[0] = n_gt;
-      cnt2[1] = n_eq;
+      cnt2[0] = static_cast<int>(total & 0xffffffffull);
+      cnt2[1] = static_cast<int>(total >> 32);
     }
   }
-  cl.sync();  // every chunk's counts are published
+  cl.sync();  // every chunk's counts are published (and this chunk's offsets are in place)
   if (tid == 0) {
     int sel_before = 0, eq_before = 0;
     for (int r = 0; r < rank; ++r) {
@@ -372,46 +380,25 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
   __syncthreads();
   const int sel_before = sh_off[0], take_eq = sh_off[1];
   const unsigned lt = (1u << lane) - 1u;
-  auto selected = [&](int j, int i) -> bool {  // warp-collective
-    if (n_route <= 0) return false;
-    if (n_route >= N) return i < n;
-    const unsigned x = i < n ? rkeys[i] : 0u;
-    const bool eq = i < n && x == T;
-    const unsigned beq = __ballot_sync(0xffffffffu, eq);
-    const int eq_rank = ceq[j * kRouteNW + w] + __popc(beq & lt);
-    return i < n && (x > T || (eq && eq_rank < take_eq));
-  };
-  for (int j = 0; j < trips; ++j) {
-    const unsigned bal = __ballot_sync(0xffffffffu, selected(j, j * kRouteCT + tid));
-    if (lane == 0) csel[j * kRouteNW + w] = __popc(bal);
-  }
-  __syncthreads();
-  {
-    const int per = (trips * kRouteNW + kRouteCT - 1) / kRouteCT;
-    int loc = 0;
-    for (int k = 0; k < per; ++k) {
-      const int e = tid * per + k;
-      if (e < trips * kRouteNW) loc += csel[e];
-    }
-    int tot;
-    int run = block_exclusive_sum_512(loc, scan_ws, tot);
-    for (int k = 0; k < per; ++k) {
-      const int e = tid * per + k;
-      if (e < trips * kRouteNW) {
-        const int c = csel[e];
-        csel[e] = run;
-        run += c;
-      }
-    }
-    __syncthreads();
-  }
   int32_t* rout = routed + static_cast<size_t>(bh) * n_route;
   int32_t* tout = taylor + static_cast<size_t>(bh) * (N - n_route);
   for (int j = 0; j < trips; ++j) {
     const int i = j * kRouteCT + tid;
-    const bool sel = selected(j, i);
-    const unsigned bal = __ballot_sync(0xffffffffu, sel);
-    const int r = sel_before + csel[j * kRouteNW + w] + __popc(bal & lt);  // routed keys before c0 + i
+    const unsigned x = i < n ? rkeys[i] : 0u;
+    bool sel;
+    int r;  // routed keys before c0 + i over the head
+    if (partial) {
+      const bool gt = i < n && x > T, eq = i < n && x == T;
+      const unsigned bgt = __ballot_sync(0xffffffffu, gt);
+      const unsigned beq = __ballot_sync(0xffffffffu, eq);
+      const int gt_b = cgt[j * kRouteNW + w] + __popc(bgt & lt);
+      const int eq_b = ceq[j * kRouteNW + w] + __popc(beq & lt);
+      sel = gt || (eq && eq_b < take_eq);
+      r = sel_before + gt_b + min(eq_b, take_eq);
+    } else {
+      sel = n_route >= N && i < n;
+      r = sel_before + (n_route >= N ? i : 0);
+    }
     if (i < n) {
       // counts are exact by construction; the guards only keep a corrupted
       // input (e.g. NaN sharpness) from writing past the buckets
