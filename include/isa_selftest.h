@@ -17,6 +17,13 @@
  * pairs as the kernels do), y_mufu = the MUFU ex2.approx.ftz used for the
  * other exponentials, y_ref = CUDA's exp2f.  Asynchronous on stream;
  * ISA_ERR_INVALID_ARG for n < 0 or a null pointer when n > 0.
+ *
+ * isa_selftest_umma_pair runs one M = 256 tile on a pair of CTAs (two SMs,
+ * one cluster): S [256, 128] fp32 = A B^T and O [256, 128] fp32 = P V with
+ * A [256, 128], B [128, 128] (keys x d), P [256, 128], V [128, 128] bf16,
+ * the even CTA issuing both products; each CTA holds 128 rows of A, half
+ * the keys of B, its 128 rows of P (in tensor memory) and half the columns
+ * of V.  ws as for isa_selftest_umma.
  */
 #ifndef ISA_SELFTEST_H_
 #define ISA_SELFTEST_H_
@@ -27,6 +34,8 @@ extern "C" {
 int isa_selftest_umma(int d, int bn, const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V,
                       float* S, float* O, float* O2, void* ws, void* stream);
 int isa_selftest_ex2(const float* x, float* y_poly, float* y_mufu, float* y_ref, int n, void* stream);
+int isa_selftest_umma_pair(const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V, float* S,
+                           float* O, void* ws, void* stream);
 #ifdef __cplusplus
 }
 #endif

@@ -63,6 +63,7 @@ SIGNATURES = {
     "isa_last_error": (ctypes.c_char_p, []),
     "isa_selftest_umma": (_I, [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "isa_selftest_ex2": (_I, [_P, _P, _P, _P, _I, _P]),
+    "isa_selftest_umma_pair": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 _lib = None

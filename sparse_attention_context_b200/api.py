@@ -361,3 +361,13 @@ def isa_selftest_ex2(x, stream=None):
     rc = lib().isa_selftest_ex2(x.data_ptr(), yp.data_ptr(), ym.data_ptr(), yr.data_ptr(), x.numel(), _stream(stream))
     check("isa_selftest_ex2", rc)
     return yp, ym, yr
+
+
+def isa_selftest_umma_pair(A, B, P, V, ws, stream=None):
+    """Test-only: one M = 256 tile on a CTA pair: S = A B^T, O = P V (fp32)."""
+    S = torch.empty((256, 128), dtype=torch.float32, device=A.device)
+    O = torch.empty((256, 128), dtype=torch.float32, device=A.device)
+    rc = lib().isa_selftest_umma_pair(A.data_ptr(), B.data_ptr(), P.data_ptr(), V.data_ptr(), S.data_ptr(),
+                                      O.data_ptr(), ws.data_ptr(), _stream(stream))
+    check("isa_selftest_umma_pair", rc)
+    return S, O

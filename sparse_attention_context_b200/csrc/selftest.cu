@@ -158,6 +158,116 @@ static int run_probe(const uint16_t* A, const uint16_t* B, const uint16_t* P, co
   return cudaGetLastError() == cudaSuccess ? ISA_OK : ISA_ERR_CUDA;
 }
 
+// One M = 256 tile on a CTA pair (cluster of 2): S = A B^T with A rows
+// [128r, 128r + 128) and B rows (keys) [64r, 64r + 64) in CTA r's shared
+// memory, then O = P V with P rows [128r, 128r + 128) in CTA r's tensor
+// memory and V columns [64r, 64r + 64) in its shared memory.  The even CTA
+// issues both products; each CTA reads its own rows of S and O back.
+// D = 128, N = 128 keys.  Operands are written into shared memory by the
+// threads (no TMA), so the probe depends on nothing but the pair UMMA.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
+    umma_pair_probe_kernel(const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V, float* S_out,
+                           float* O_out, int* status) {
+  constexpr int D = 128, BN = 128;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  uint8_t* sA = smem;                       // 128 rows x 128 d, K-major: 2 chunks of 16 KB
+  uint8_t* sB = sA + 128 * D * 2;           // 64 keys x 128 d, K-major: 2 chunks of 8 KB
+  uint8_t* sV = sB + 64 * D * 2;            // 128 keys x 64 d, MN-major: 16 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 128 * 64 * 2);  // [0] S done, [1] O done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  constexpr int PCOL = 256, OCOL = 128;     // S at [0, 128), O at [128, 256), P at [256, 320)
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t rank = cluster_ctarank();
+
+  for (int c = tid; c < 128 * (D / 8); c += 128) {
+    const int row = c / (D / 8), ch = c % (D / 8);
+    const uint4 val = *reinterpret_cast<const uint4*>(A + (128 * rank + row) * D + ch * 8);
+    st_shared_v4(smem_u32(sA) + (ch >> 3) * (128 * 128) + sw128(row, ch & 7), val.x, val.y, val.z, val.w);
+  }
+  for (int c = tid; c < 64 * (D / 8); c += 128) {
+    const int row = c / (D / 8), ch = c % (D / 8);
+    const uint4 val = *reinterpret_cast<const uint4*>(B + (64 * rank + row) * D + ch * 8);
+    st_shared_v4(smem_u32(sB) + (ch >> 3) * (64 * 128) + sw128(row, ch & 7), val.x, val.y, val.z, val.w);
+  }
+  for (int c = tid; c < BN * 8; c += 128) {
+    const int key = c / 8, ch = c % 8;
+    const uint4 val = *reinterpret_cast<const uint4*>(V + key * D + 64 * rank + ch * 8);
+    st_shared_v4(smem_u32(sV) + sw128(key, ch), val.x, val.y, val.z, val.w);
+  }
+  fence_proxy_async_smem();
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int row = tid;
+  const uint32_t lb = static_cast<uint32_t>(warp * 32) << 16;
+  // P rows of this CTA into TMEM: column c holds P[row][2c] (low half), P[row][2c+1]
+#pragma unroll
+  for (int j = 0; j < BN / 64; ++j) {
+    uint32_t u[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      u[i] = static_cast<uint32_t>(P[(128 * rank + row) * BN + j * 64 + 2 * i]) |
+             (static_cast<uint32_t>(P[(128 * rank + row) * BN + j * 64 + 2 * i + 1]) << 16);
+    tmem_st32(tmem + lb + PCOL + j * 32, u);
+  }
+  tmem_wait_st();
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' operands, barriers and TMEM in place
+  tc_fence_after();
+  if (rank == 0 && tid == 0) {
+    constexpr uint32_t IDS = idesc_bf16(256, BN, 0);
+    constexpr uint32_t IDO = idesc_bf16(256, D, 1);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      umma_pair_bf16(tmem, desc_k_sw128(smem_u32(sA) + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                     desc_k_sw128(smem_u32(sB) + (kk >> 2) * (64 * 128) + (kk & 3) * 32), IDS, kk > 0 ? 1u : 0u);
+    umma_commit_pair(&bars[0], 3);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk)
+      umma_pair_bf16_tmem_a(tmem + OCOL, tmem + PCOL + kk * 8, desc_mn_sw128(smem_u32(sV) + kk * 16 * 128, 128 * 128),
+                            IDO, kk > 0 ? 1u : 0u);
+    umma_commit_pair(&bars[1], 3);
+  }
+  __syncwarp();
+  bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[0], 0, nullptr, kWaitLimitNs) == 0);
+  ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(&bars[1], 0, nullptr, kWaitLimitNs) == 0);
+  tc_fence_after();
+  if (ok) {
+    for (int j = 0; j < BN / 32; ++j) {
+      uint32_t u[32];
+      tmem_ld32(tmem + lb + j * 32, u);
+      tmem_wait_ld();
+      for (int i = 0; i < 32; ++i) S_out[(128 * rank + row) * BN + j * 32 + i] = __uint_as_float(u[i]);
+    }
+    for (int j = 0; j < D / 32; ++j) {
+      uint32_t u[32];
+      tmem_ld32(tmem + lb + OCOL + j * 32, u);
+      tmem_wait_ld();
+      for (int i = 0; i < 32; ++i) O_out[(128 * rank + row) * D + j * 32 + i] = __uint_as_float(u[i]);
+    }
+  } else if (tid == 0) {
+    atomicCAS(status, 0, ISA_ERR_DEVICE_TIMEOUT);
+  }
+  tc_fence_before();
+  cluster_sync_all();  // neither CTA frees TMEM or exits while the pair's UMMAs or reads run
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 // y_poly = ex2_poly2(x) (two arguments per call, as the softmax uses it),
 // y_mufu = ex2.approx.ftz (the MUFU path), y_ref = exp2f; one thread per pair.
 __global__ void __launch_bounds__(256) ex2_probe_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
@@ -187,6 +297,19 @@ extern "C" int isa_selftest_ex2(const float* x, float* y_poly, float* y_mufu, fl
   const int pairs = (n + 1) / 2;
   isa::ex2_probe_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_mufu,
                                                                                             y_ref, n);
+  return isa::record_cuda_status(cudaGetLastError());
+}
+
+extern "C" int isa_selftest_umma_pair(const uint16_t* A, const uint16_t* B, const uint16_t* P, const uint16_t* V,
+                                      float* S, float* O, void* ws, void* stream) {
+  if (!A || !B || !P || !V || !S || !O || !ws) return ISA_ERR_INVALID_ARG;
+  const int smem = 128 * 128 * 2 + 64 * 128 * 2 + 128 * 64 * 2 + 64 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(isa::umma_pair_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       116 * 1024);  // one CTA per SM: each pair CTA holds all 512 TMEM columns
+  if (e != cudaSuccess) return isa::record_cuda_status(e);
+  (void)smem;
+  isa::umma_pair_probe_kernel<<<2, 128, 116 * 1024, static_cast<cudaStream_t>(stream)>>>(A, B, P, V, S, O,
+                                                                                         static_cast<int*>(ws));
   return isa::record_cuda_status(cudaGetLastError());
 }
 

@@ -25,3 +25,22 @@ def test_umma_tile(cuda_ok, d, bn):
     assert torch.allclose(S.cpu().double(), S_ref, rtol=1e-5, atol=1e-4), (S.cpu().double() - S_ref).abs().max()
     assert torch.allclose(O.cpu().double(), O_ref, rtol=1e-5, atol=1e-4), (O.cpu().double() - O_ref).abs().max()
     assert torch.allclose(O2.cpu().double(), O_ref, rtol=1e-5, atol=1e-4), (O2.cpu().double() - O_ref).abs().max()
+
+
+def test_umma_pair_tile(cuda_ok):
+    """One M = 256 tile on a CTA pair (cta_group::2): each CTA holds 128 rows
+    of A, half the keys of B and half the columns of V; both products must
+    equal the float64 ones row for row."""
+    g = torch.Generator().manual_seed(2561)
+    A = torch.randn(256, 128, generator=g).bfloat16()
+    B = torch.randn(128, 128, generator=g).bfloat16()
+    P = torch.rand(256, 128, generator=g).bfloat16()
+    V = torch.randn(128, 128, generator=g).bfloat16()
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    S, O = api.isa_selftest_umma_pair(A.cuda(), B.cuda(), P.cuda(), V.cuda(), ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    S_ref = A.double() @ B.double().T
+    O_ref = P.double() @ V.double()
+    assert torch.allclose(S.cpu().double(), S_ref, rtol=1e-5, atol=1e-4), (S.cpu().double() - S_ref).abs().max()
+    assert torch.allclose(O.cpu().double(), O_ref, rtol=1e-5, atol=1e-4), (O.cpu().double() - O_ref).abs().max()
