@@ -263,10 +263,8 @@ int run_full_rows(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint
   const Dims& d = c.d;
   cudaError_t e = cudaSuccess;
   if (n_rows > 0) {
-    const bool pair = attn_pair_supported(d.d, d.blk);
     CUtensorMap tmK, tmV;
-    // the pair engine loads half a key tile per CTA (box of blk/2 rows)
-    if (!make_tmap_bf16(&tmK, k, static_cast<uint64_t>(d.BH) * d.N, d.d, pair ? d.blk / 2 : d.blk) ||
+    if (!make_tmap_bf16(&tmK, k, static_cast<uint64_t>(d.BH) * d.N, d.d, d.blk) ||
         !make_tmap_bf16(&tmV, v, static_cast<uint64_t>(d.BH) * d.N, d.d, d.blk))
       return ISA_ERR_CUDA;
     FlashParams p = base_params(c);
@@ -277,8 +275,7 @@ int run_full_rows(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint
     p.kept_ctx = kept;
     p.n_kv_tiles = d.nSB + d.n_keep;
     p.kv_rows_per_head = d.N;
-    e = pair ? launch_attn_pair(MODE_FULL, tmK /* Q is gathered by threads */, tmK, tmV, p, d.BH, c.st)
-             : launch_attn2(d.d, d.blk, MODE_FULL, tmK /* Q is gathered by threads */, tmK, tmV, p, d.BH, c.st);
+    e = launch_attn2(d.d, d.blk, MODE_FULL, tmK /* Q is gathered by threads */, tmK, tmV, p, d.BH, c.st);
   }
   return cuda_status(e);
 }
@@ -673,10 +670,9 @@ int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* 
   // key-split partials after the control block, as many CTAs as fit
   const size_t per = split_bytes_per_cta(d);
   const int cap = ws_bytes > kCtlBytes + 4096 ? static_cast<int>((ws_bytes - kCtlBytes - 4096) / per) : 0;
-  const bool pair = attn_pair_supported(d, 128);
   CUtensorMap tmQ, tmK, tmV;
   if (!make_tmap_bf16(&tmQ, q, static_cast<uint64_t>(BH) * N, d, 128) ||
-      !make_tmap_bf16(&tmK, k, static_cast<uint64_t>(BH) * N, d, pair ? 64 : 128) ||
+      !make_tmap_bf16(&tmK, k, static_cast<uint64_t>(BH) * N, d, 128) ||
       !make_tmap_bf16(&tmV, v, static_cast<uint64_t>(BH) * N, d, 128))
     return ISA_ERR_CUDA;
   FlashParams p{};
@@ -695,9 +691,6 @@ int isa_dense_attn_fwd(int B, int H, int N, int d, float scale, const uint16_t* 
     p.ml_part = at<float2>(ws, align256(kCtlBytes + static_cast<size_t>(cap) * 256 * d * 4));
     p.split_capacity = cap;
   }
-  if (pair)
-    return cuda_status(
-        launch_attn_pair(MODE_DENSE, tmQ, tmK, tmV, p, static_cast<int>(BH), static_cast<cudaStream_t>(stream)));
   return cuda_status(launch_attn2(d, 128, MODE_DENSE, tmQ, tmK, tmV, p, static_cast<int>(BH),
                                   static_cast<cudaStream_t>(stream)));
 }

@@ -96,13 +96,6 @@ cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi
                          cudaStream_t st);
 cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                          const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st);
-// The same engine on SM pairs (flash_pair.cu, cta_group::2 UMMAs of M =
-// 256), for D = 128 and 128-key tiles: 512-row work items per pair, the
-// key-split tail over pairs.  tmQ as above (box 128 rows), tmKh over K with
-// box 64 rows (a key half), tmV over V with box 128 rows.
-bool attn_pair_supported(int D, int BN);
-cudaError_t launch_attn_pair(int mode, const CUtensorMap& tmQ, const CUtensorMap& tmKh, const CUtensorMap& tmV,
-                             const FlashParams& p, int BH, cudaStream_t st);
 
 // Stage-1 kernels.
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,
