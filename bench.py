@@ -64,15 +64,17 @@ def counts(cfg):
 
 # DRAM bytes (read + write) of one routed full-attention stage at the 480p
 # workload -- whole-wave launch, key-split launch and combine -- summed from
-# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass).
+# ncu captures of one kernel each (dram__bytes_read.sum +
+# dram__bytes_write.sum, one pass).
 # They hold only for the kernel sources they were taken on: on any other
 # source, or another workload, the report's traffic is null.
 FULL_TRAFFIC = {
     "config": "480p",
-    "bytes": 384_441_088 + 36_827_392 + 14_966_272 + 768 + 18_468_864,
+    # whole-wave launch (read + write), key-split launch (read + write), combine
+    "bytes": 398_867_456 + 40_851_456 + 14_972_672 + 8_448 + 18_467_840 + 0,
     "sources": {
-        "sparse_attention_context_b200/csrc/flash2.cu": "88a1e0b4f250bdc90e7b7e9834951c272f145ee77aabc0ae46734358e9a49539",
-        "sparse_attention_context_b200/csrc/tc_ptx.cuh": "a99eac8f56d3542436ffd184ac1c8e2e863e048d2eef2dcbc2189b53b0161f21",
+        "sparse_attention_context_b200/csrc/flash2.cu": "fb5e1c53903090b2ec4ec14ea27383a3a30a47cbc8eb67d22a5b2b6505ba355c",
+        "sparse_attention_context_b200/csrc/tc_ptx.cuh": "1026ba5d3e08b740b9d4aa8f4fc7e2bd31b8c482744693570e460f8679e5be71",
     },
 }
 
