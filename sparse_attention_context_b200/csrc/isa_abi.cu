@@ -18,13 +18,13 @@ namespace isa {
 namespace {
 
 struct Dims {
-  int B, H, BH, N_src, N_ctx, N, d, blk, nSB, nCB, nB, n_keep, n_route, n_rb, nK, nKpad, nChunks;
+  int B, H, BH, N_src, N_ctx, N, d, blk, nSB, nCB, nB, nBp, n_keep, n_route, n_rb, nK, nKpad, nChunks;
   float scale;
 };
 
 struct WsLayout {
-  size_t Qbar, Kbar, Vbar, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, rblk, rrows, opart, mlpart,
-      total;
+  size_t Kbar, Vbar, qksplit, salstats, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, rblk,
+      rrows, opart, mlpart, total;
   int split_ctas;  // key-split partial CTAs the workspace holds
 };
 
@@ -82,7 +82,8 @@ int check_shape(const isa_shape* s, Dims* o) {
   d.n_rb = route_count(s->rho, d.nB);  // block-granular grouping: same rule over the nB query blocks
   d.nK = d.nSB + d.n_keep;
   d.nKpad = (d.nK + 127) / 128 * 128;
-  d.nChunks = (d.nB + kSalRows - 1) / kSalRows;
+  d.nBp = (d.nB + 127) / 128 * 128;
+  d.nChunks = d.nBp / 128;  // saliency row tiles
   d.scale = s->scale > 0.f ? s->scale : 1.0f / std::sqrt(static_cast<float>(d.d));
   *o = d;
   return ISA_OK;
@@ -97,9 +98,10 @@ WsLayout layout(const Dims& d) {
     return at;
   };
   const size_t BH = d.BH;
-  L.Qbar = take(BH * d.nB * d.d * 4);
   L.Kbar = take(BH * d.nB * d.d * 4);
   L.Vbar = take(BH * d.nB * d.d * 4);
+  L.qksplit = take(4 * BH * d.nBp * d.d * 2);
+  L.salstats = take(BH * d.nChunks * d.nBp * 8);
   L.partial = take(BH * d.nChunks * std::max(d.nCB, 1) * 4);
   L.sal = take(BH * std::max(d.nCB, 1) * 4);
   L.Khi = take(BH * d.nKpad * d.d * 2);
@@ -182,14 +184,17 @@ FlashParams base_params(const Ctx& c) {
 int run_preselect(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint16_t* v, int32_t* kept,
                   float* sal_user) {
   const Dims& d = c.d;
-  cudaError_t e = launch_pool(q, k, v, at<float>(c.ws, c.L.Qbar), at<float>(c.ws, c.L.Kbar),
-                              at<float>(c.ws, c.L.Vbar), d.BH, d.N_src, d.N_ctx, d.d, d.blk, c.st);
+  uint16_t* split = at<uint16_t>(c.ws, c.L.qksplit);
+  const size_t plane = static_cast<size_t>(d.BH) * d.nBp * d.d;  // Qhi, Qlo, Khi, Klo
+  cudaError_t e = launch_pool(q, k, v, nullptr, at<float>(c.ws, c.L.Kbar),
+                              at<float>(c.ws, c.L.Vbar), split, d.BH, d.N_src, d.N_ctx, d.d, d.blk, c.st);
   if (e == cudaSuccess)
-    e = launch_saliency(at<float>(c.ws, c.L.Qbar), at<float>(c.ws, c.L.Kbar), at<float>(c.ws, c.L.partial), d.BH,
-                        d.N_src, d.N_ctx, d.d, d.blk, d.scale, c.st);
+    e = launch_saliency_tc(split, split + plane, split + 2 * plane, split + 3 * plane,
+                           at<float2>(c.ws, c.L.salstats), at<float>(c.ws, c.L.partial), d.BH, d.N_src, d.N_ctx,
+                           d.d, d.blk, d.scale, c.status(), c.st);
   if (e == cudaSuccess)
-    e = launch_select_ctx(at<float>(c.ws, c.L.partial), at<float>(c.ws, c.L.sal), sal_user, kept, d.BH, d.N_src,
-                          d.N_ctx, d.blk, d.n_keep, c.st);
+    e = launch_select_ctx(at<float>(c.ws, c.L.partial), d.nChunks, at<float>(c.ws, c.L.sal), sal_user, kept, d.BH,
+                          d.N_src, d.N_ctx, d.blk, d.n_keep, c.st);
   return cuda_status(e);
 }
 

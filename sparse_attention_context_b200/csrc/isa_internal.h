@@ -13,7 +13,6 @@ constexpr int kStatusOffset = 0;   // int32 in the workspace control block
 constexpr int kInjectOffset = 4;   // int32 fault-injection word (tests)
 constexpr int kCtlBytes = 256;
 constexpr int kTopkCap = 4096;     // max context blocks the top-k sort holds
-constexpr int kSalRows = 32;       // query blocks per saliency CTA
 constexpr int kRouteBlocksCap = 16384;  // max query blocks per head of the block grouping
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
@@ -97,13 +96,20 @@ cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi
 cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                          const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st);
 
-// Stage-1 kernels.
+// Stage-1 kernels.  launch_pool writes fp32 Kbar and Vbar (Qbar too unless
+// it is null) and bf16 hi / lo of Qbar and Kbar
+// into QKsplit: four [BH, nBp, D] arrays (Qhi, Qlo, Khi, Klo), nBp = nB
+// rounded up to 128, pad rows left unwritten.  launch_saliency_tc: partial
+// [BH, nBp/128, nCB] column sums per 128-row tile (stats [BH, nBp/128, nBp]
+// float2 scratch); launch_select_ctx adds the n_chunks partial rows in order.
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,
-                        float* Vbar, int BH, int N_src, int N_ctx, int D, int blk, cudaStream_t st);
-cudaError_t launch_saliency(const float* Qbar, const float* Kbar, float* partial, int BH, int N_src, int N_ctx,
-                            int D, int blk, float scale, cudaStream_t st);
-cudaError_t launch_select_ctx(const float* partial, float* sal_ws, float* sal_user, int32_t* kept, int BH,
-                              int N_src, int N_ctx, int blk, int n_keep, cudaStream_t st);
+                        float* Vbar, uint16_t* QKsplit, int BH, int N_src, int N_ctx, int D, int blk,
+                        cudaStream_t st);
+cudaError_t launch_saliency_tc(const uint16_t* Qhi, const uint16_t* Qlo, const uint16_t* Khi, const uint16_t* Klo,
+                               float2* stats, float* partial, int BH, int N_src, int N_ctx, int D, int blk,
+                               float scale, int* status, cudaStream_t st);
+cudaError_t launch_select_ctx(const float* partial, int n_chunks, float* sal_ws, float* sal_user, int32_t* kept,
+                              int BH, int N_src, int N_ctx, int blk, int n_keep, cudaStream_t st);
 cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_t* kept, uint16_t* Khi,
                               uint16_t* Klo, uint16_t* Vb, float* bias2, int BH, int N_src, int N_ctx, int D,
                               int blk, int n_keep, int nKpad, int* status, cudaStream_t st);

@@ -9,6 +9,8 @@
 // chunk over a strided set of rows, then the row groups' partial sums are
 // added through shared memory.  HBM-bound: every byte of q, k, v is read
 // once.
+#include <cuda_bf16.h>
+
 #include "isa_internal.h"
 #include "tc_ptx.cuh"
 
@@ -26,12 +28,18 @@ __device__ __forceinline__ void acc_bf16x8(float (&a)[8], const uint4& w) {
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                                                    const uint16_t* __restrict__ v, float* __restrict__ Qbar,
-                                                   float* __restrict__ Kbar, float* __restrict__ Vbar, int N_src,
-                                                   int N_ctx, int blk, int nSB, int nB) {
+                                                   float* __restrict__ Kbar, float* __restrict__ Vbar,
+                                                   uint16_t* __restrict__ QKsplit, int N_src, int N_ctx, int blk,
+                                                   int nSB, int nB, int nBp) {
   constexpr int CPR = D / 8;          // 16-byte chunks per row
   constexpr int RG = 256 / CPR;       // row groups (rows in flight per pass)
   __shared__ float red[3][RG][D + 4];
   const int b = blockIdx.x, bh = blockIdx.y;
+  // bf16 hi + lo of Qbar and Kbar for the tensor-core saliency: four
+  // [BH, nBp, D] arrays (Qhi, Qlo, Khi, Klo); rows nB..nBp-1 are not written
+  // (the saliency kernel masks them)
+  const size_t split_plane = static_cast<size_t>(gridDim.y) * nBp * D;
+  uint16_t* split_row = QKsplit + (static_cast<size_t>(bh) * nBp + b) * D;
   const int N = N_src + N_ctx;
   const int start = b < nSB ? b * blk : N_src + (b - nSB) * blk;
   const int cnt = b < nSB ? min(blk, N_src - b * blk) : min(blk, N_ctx - (b - nSB) * blk);
@@ -61,20 +69,29 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
     float s = 0.f;
 #pragma unroll
     for (int g = 0; g < RG; ++g) s += red[t][g][col];
-    float* dst = t == 0 ? Qbar : (t == 1 ? Kbar : Vbar);
-    dst[(static_cast<size_t>(bh) * nB + b) * D + col] = s / fcnt;
+    const float mean = s / fcnt;
+    float* dst = t == 0 ? Qbar : (t == 1 ? Kbar : Vbar);  // Qbar may be null: only its bf16 split is used
+    if (dst != nullptr) dst[(static_cast<size_t>(bh) * nB + b) * D + col] = mean;
+    if (t < 2) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(mean - __bfloat162float(hi));
+      split_row[(2 * t) * split_plane + col] = __bfloat16_as_ushort(hi);
+      split_row[(2 * t + 1) * split_plane + col] = __bfloat16_as_ushort(lo);
+    }
   }
 }
 
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,
-                        float* Vbar, int BH, int N_src, int N_ctx, int D, int blk, cudaStream_t st) {
+                        float* Vbar, uint16_t* QKsplit, int BH, int N_src, int N_ctx, int D, int blk,
+                        cudaStream_t st) {
   const int nSB = (N_src + blk - 1) / blk, nCB = (N_ctx + blk - 1) / blk;
   const int nB = nSB + nCB;
+  const int nBp = (nB + 127) / 128 * 128;
   const dim3 grid(nB, BH);
   if (D == 128)
-    pool_kernel<128><<<grid, 256, 0, st>>>(q, k, v, Qbar, Kbar, Vbar, N_src, N_ctx, blk, nSB, nB);
+    pool_kernel<128><<<grid, 256, 0, st>>>(q, k, v, Qbar, Kbar, Vbar, QKsplit, N_src, N_ctx, blk, nSB, nB, nBp);
   else
-    pool_kernel<64><<<grid, 256, 0, st>>>(q, k, v, Qbar, Kbar, Vbar, N_src, N_ctx, blk, nSB, nB);
+    pool_kernel<64><<<grid, 256, 0, st>>>(q, k, v, Qbar, Kbar, Vbar, QKsplit, N_src, N_ctx, blk, nSB, nB, nBp);
   return cudaGetLastError();
 }
 
