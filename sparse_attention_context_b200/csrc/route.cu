@@ -240,8 +240,12 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
   int* cgt = reinterpret_cast<int*>(rkeys + chunk);          // [trips][NW] keys > T, then their offsets
   int* ceq = cgt + trips * kRouteNW;                         // [trips][NW] keys == T, then their offsets
   __shared__ int whist[kRouteNW][257];                       // per warp, padded
-  __shared__ int hist[2][256];                               // this chunk's histogram, by pass parity
-  __shared__ int cnt2[2];                                    // keys > T, keys == T of this chunk
+  // every chunk's histogram, pushed by its CTA into all CTAs of the cluster
+  // (remote stores before the cluster barrier; local reads after it), by
+  // pass parity
+  __shared__ int hist_all[2][kRouteCluster][256];
+  __shared__ int tot[256];                                   // cluster-wide histogram of the pass
+  __shared__ int cnt_all[kRouteCluster][2];                  // every chunk's keys > T, keys == T (pushed)
   __shared__ unsigned sh_sel[2];                             // each pass's decision, by pass parity
   __shared__ int sh_rem[2];
   __shared__ int sh_off[2];                                  // routed keys before this chunk, equal keys it takes
@@ -278,22 +282,31 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
           t += whist[ww][tid];
           whist[ww][tid] = 0;
         }
-        hist[buf][tid] = t;
+        const uint32_t mine = static_cast<uint32_t>(__cvta_generic_to_shared(&hist_all[buf][rank][tid]));
+#pragma unroll
+        for (int r = 0; r < kRouteCluster; ++r)
+          asm volatile("{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\tst.shared::cluster.u32 [ra], %2;\n\t}" ::"r"(mine), "r"(r), "r"(t)
+                       : "memory");
       }
+      // every chunk's histogram of this pass has arrived everywhere (and every
+      // read of the other buffer, two passes back, is done)
       cl.sync();
+      if (tid < 256) {
+        int t = 0;
+#pragma unroll
+        for (int r = 0; r < kRouteCluster; ++r) t += hist_all[buf][r][tid];
+        tot[tid] = t;
+      }
+      __syncthreads();
       if (w == 0) {
-        // lane l owns bins 255-8l .. 248-8l (descending): the cluster-wide
-        // counts, then the bin where the count from the top reaches `remaining`
-        int tot[8];
+        // lane l owns bins 255-8l .. 248-8l (descending): the bin where the
+        // count from the top reaches `remaining`
+        int tl[8];
         int s = 0;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const int bin = 255 - 8 * lane - k;
-          int t = 0;
-#pragma unroll
-          for (int r = 0; r < kRouteCluster; ++r) t += cl.map_shared_rank(&hist[buf][0], r)[bin];
-          tot[k] = t;
-          s += t;
+          tl[k] = tot[255 - 8 * lane - k];
+          s += tl[k];
         }
         int incl = s;
 #pragma unroll
@@ -306,12 +319,12 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
           int cum = before;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            if (cum + tot[k] >= remaining) {
+            if (cum + tl[k] >= remaining) {
               sh_sel[buf] = static_cast<unsigned>(255 - 8 * lane - k);
               sh_rem[buf] = remaining - cum;
               break;
             }
-            cum += tot[k];
+            cum += tl[k];
           }
         }
       }
@@ -360,22 +373,23 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
         run += static_cast<unsigned long long>(g) | (static_cast<unsigned long long>(q) << 32);
       }
     }
-    if (tid == 0) {
-      cnt2[0] = static_cast<int>(total & 0xffffffffull);
-      cnt2[1] = static_cast<int>(total >> 32);
+    if (tid < kRouteCluster) {  // this chunk's counts into every CTA of the cluster
+      const uint32_t mine = static_cast<uint32_t>(__cvta_generic_to_shared(&cnt_all[rank][0]));
+      const int g = static_cast<int>(total & 0xffffffffull), q = static_cast<int>(total >> 32);
+      asm volatile("{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\tst.shared::cluster.v2.u32 [ra], {%2, %3};\n\t}" ::"r"(mine), "r"(tid), "r"(g), "r"(q)
+                   : "memory");
     }
   }
-  cl.sync();  // every chunk's counts are published (and this chunk's offsets are in place)
+  cl.sync();  // every chunk's counts have arrived (and this chunk's offsets are in place)
   if (tid == 0) {
     int sel_before = 0, eq_before = 0;
     for (int r = 0; r < rank; ++r) {
-      const int* cr = cl.map_shared_rank(&cnt2[0], r);
-      const int r_gt = cr[0], r_eq = cr[1];
+      const int r_gt = cnt_all[r][0], r_eq = cnt_all[r][1];
       sel_before += r_gt + min(r_eq, max(0, need_eq - eq_before));
       eq_before += r_eq;
     }
     sh_off[0] = n_route >= N ? c0 : (n_route <= 0 ? 0 : sel_before);
-    sh_off[1] = min(cnt2[1], max(0, need_eq - eq_before));  // equal keys of this chunk that are routed
+    sh_off[1] = min(cnt_all[rank][1], max(0, need_eq - eq_before));  // equal keys of this chunk that are routed
   }
   __syncthreads();
   const int sel_before = sh_off[0], take_eq = sh_off[1];
@@ -412,7 +426,7 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteCT
       }
     }
   }
-  cl.sync();  // peers may still read this CTA's counts until here
+  cl.sync();  // no CTA exits while a peer may still store into it
 }
 
 cudaError_t launch_route(const float* sharp, int32_t* routed, int32_t* taylor, int BH, int N, int n_route,
