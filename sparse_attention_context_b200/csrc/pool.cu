@@ -64,19 +64,26 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
   }
   __syncthreads();
   const float fcnt = static_cast<float>(cnt);
-  for (int e = threadIdx.x; e < 3 * D; e += 256) {
-    const int t = e / D, col = e % D;
-    float s = 0.f;
+  // two adjacent columns per thread: 8-byte fp32 and 4-byte bf16x2 stores
+  for (int e = threadIdx.x; e < 3 * D / 2; e += 256) {
+    const int t = (2 * e) / D, col = (2 * e) % D;
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int g = 0; g < RG; ++g) s += red[t][g][col];
-    const float mean = s / fcnt;
+    for (int g = 0; g < RG; ++g) {
+      s0 += red[t][g][col];
+      s1 += red[t][g][col + 1];
+    }
+    const float m0 = s0 / fcnt, m1 = s1 / fcnt;
     float* dst = t == 0 ? Qbar : (t == 1 ? Kbar : Vbar);  // Qbar may be null: only its bf16 split is used
-    if (dst != nullptr) dst[(static_cast<size_t>(bh) * nB + b) * D + col] = mean;
+    if (dst != nullptr) *reinterpret_cast<float2*>(dst + (static_cast<size_t>(bh) * nB + b) * D + col) = make_float2(m0, m1);
     if (t < 2) {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(mean - __bfloat162float(hi));
-      split_row[(2 * t) * split_plane + col] = __bfloat16_as_ushort(hi);
-      split_row[(2 * t + 1) * split_plane + col] = __bfloat16_as_ushort(lo);
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(m0), h1 = __float2bfloat16_rn(m1);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(m0 - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(m1 - __bfloat162float(h1));
+      *reinterpret_cast<uint32_t*>(split_row + (2 * t) * split_plane + col) =
+          static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+      *reinterpret_cast<uint32_t*>(split_row + (2 * t + 1) * split_plane + col) =
+          static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
     }
   }
 }
