@@ -568,6 +568,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--heads", type=int, default=None, help="override H (small profiling captures)")
     ap.add_argument("--rho", type=float, default=None, help="override rho (profiling captures)")
     ap.add_argument("--keep", type=float, default=None, help="override keep (profiling captures)")
@@ -696,6 +697,33 @@ def main():
     ms_max = max_over_ranks(ms, dev)
     assert api.isa_read_device_status(ws) == 0
 
+    # the same step captured once in a CUDA graph and replayed (the launch
+    # sequence without host calls between kernels); reported beside `value`
+    graph_ms = None
+    if not args.no_graph:
+        gs = torch.cuda.Stream()
+        gs.wait_stream(stream)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gs):
+            api.isa_preselect_ctx(q, k, v, shape, ws, kept=kept, want_saliency=False, stream=gs)
+            api.isa_route_taylor_fwd(q, kept, shape, ws, out, routed=routed, taylor=taylor, want_sharpness=False,
+                                     stream=gs)
+            api.isa_full_attn_fwd(q, k, v, kept, routed, shape, ws, out, stream=gs)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps, dev)
+        assert api.isa_read_device_status(ws) == 0
+        del graph
+
     # in-house dense kernel on the same inputs (the baseline the metric names)
     dense_ms = None
     if not args.no_dense:
@@ -798,6 +826,7 @@ def main():
                             "sharpness_taylor_route": round(float(stage_ms[1]), 4),
                             "full_attn": round(float(stage_ms[2]), 4)},
                "executed_tflop": round((wm["full_flops"] + wm["fused_flops"]) / 1e12, 4),
+               "graph_ms": None if graph_ms is None else round(graph_ms, 4),
                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary()}
         if gather_ms is not None:
