@@ -23,7 +23,7 @@ struct Dims {
 };
 
 struct WsLayout {
-  size_t Kbar, Vbar, qksplit, salstats, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, rblk,
+  size_t Kbar, Vbar, qksplit, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, rblk,
       rrows, opart, mlpart, total;
   int split_ctas;  // key-split partial CTAs the workspace holds
 };
@@ -101,7 +101,6 @@ WsLayout layout(const Dims& d) {
   L.Kbar = take(BH * d.nB * d.d * 4);
   L.Vbar = take(BH * d.nB * d.d * 4);
   L.qksplit = take(4 * BH * d.nBp * d.d * 2);
-  L.salstats = take(BH * d.nChunks * d.nBp * 8);
   L.partial = take(BH * d.nChunks * std::max(d.nCB, 1) * 4);
   L.sal = take(BH * std::max(d.nCB, 1) * 4);
   L.Khi = take(BH * d.nKpad * d.d * 2);
@@ -190,8 +189,8 @@ int run_preselect(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint
                               at<float>(c.ws, c.L.Vbar), split, d.BH, d.N_src, d.N_ctx, d.d, d.blk, c.st);
   if (e == cudaSuccess)
     e = launch_saliency_tc(split, split + plane, split + 2 * plane, split + 3 * plane,
-                           at<float2>(c.ws, c.L.salstats), at<float>(c.ws, c.L.partial), d.BH, d.N_src, d.N_ctx,
-                           d.d, d.blk, d.scale, c.status(), c.st);
+                           at<float>(c.ws, c.L.partial), d.BH, d.N_src, d.N_ctx, d.d, d.blk, d.scale, c.status(),
+                           c.st);
   if (e == cudaSuccess)
     e = launch_select_ctx(at<float>(c.ws, c.L.partial), d.nChunks, at<float>(c.ws, c.L.sal), sal_user, kept, d.BH,
                           d.N_src, d.N_ctx, d.blk, d.n_keep, c.st);

@@ -100,14 +100,14 @@ cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const 
 // it is null) and bf16 hi / lo of Qbar and Kbar
 // into QKsplit: four [BH, nBp, D] arrays (Qhi, Qlo, Khi, Klo), nBp = nB
 // rounded up to 128, pad rows left unwritten.  launch_saliency_tc: partial
-// [BH, nBp/128, nCB] column sums per 128-row tile (stats [BH, nBp/128, nBp]
-// float2 scratch); launch_select_ctx adds the n_chunks partial rows in order.
+// [BH, nBp/128, nCB] column sums per 128-row tile; launch_select_ctx adds
+// the n_chunks partial rows in order.
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,
                         float* Vbar, uint16_t* QKsplit, int BH, int N_src, int N_ctx, int D, int blk,
                         cudaStream_t st);
 cudaError_t launch_saliency_tc(const uint16_t* Qhi, const uint16_t* Qlo, const uint16_t* Khi, const uint16_t* Klo,
-                               float2* stats, float* partial, int BH, int N_src, int N_ctx, int D, int blk,
-                               float scale, int* status, cudaStream_t st);
+                               float* partial, int BH, int N_src, int N_ctx, int D, int blk, float scale,
+                               int* status, cudaStream_t st);
 cudaError_t launch_select_ctx(const float* partial, int n_chunks, float* sal_ws, float* sal_user, int32_t* kept,
                               int BH, int N_src, int N_ctx, int blk, int n_keep, cudaStream_t st);
 cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_t* kept, uint16_t* Khi,
