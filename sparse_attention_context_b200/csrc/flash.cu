@@ -29,6 +29,7 @@
 // in-flight copies and MMAs, frees TMEM and returns.
 #include <cmath>
 
+#include "gather.cuh"
 #include "isa_internal.h"
 #include "tc_ptx.cuh"
 
@@ -255,23 +256,8 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------- Q load, softmax, epilogue
-    constexpr int CPR = D / 8;  // 16-byte chunks per row
     const int r0 = tile * 128;
-#pragma unroll 4
-    for (int it = 0; it < CPR; ++it) {
-      const int c = it * 128 + tid;
-      const int row = c / CPR, ch = c % CPR;
-      const int g = r0 + row;
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (g < p.n_rows) {
-        const int src = p.row_idx ? __ldg(p.row_idx + static_cast<size_t>(bh) * p.n_rows + g) : g;
-        if (static_cast<unsigned>(src) < static_cast<unsigned>(p.N))
-          val = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.N + src) * D + ch * 8));
-        else if (p.status != nullptr)
-          atomicCAS(p.status, 0, 1 /* ISA_ERR_INVALID_ARG: index out of range, row skipped */);
-      }
-      st_shared_v4(aQ + (ch >> 3) * (128 * 128) + sw128(row, ch & 7), val.x, val.y, val.z, val.w);
-    }
+    gather_rows_sw128<D>(p.q, p.row_idx, bh, p.n_rows, p.N, r0, tid, aQ, false, p.status);
     fence_proxy_async_smem();
     mbar_arrive(&bars->q_full);
 

@@ -43,6 +43,7 @@
 
 #include <cmath>
 
+#include "gather.cuh"
 #include "isa_internal.h"
 #include "tc_ptx.cuh"
 
@@ -430,29 +431,7 @@ __global__ void __launch_bounds__(320, 1)
     const int g = row0 + i * 128 + r;
     {
       // gather the tile's query rows into shared memory (K-major, 128B swizzle)
-      constexpr int CPR = D / 8;
-      uint4 vals[CPR];
-#pragma unroll
-      for (int it = 0; it < CPR; ++it) {
-        const int c = it * 128 + r;
-        const int row = c / CPR, ch = c % CPR;
-        const int gg = row0 + i * 128 + row;
-        vals[it] = make_uint4(0u, 0u, 0u, 0u);
-        if (gg < p.n_rows) {
-          const int src = p.row_idx ? __ldg(p.row_idx + static_cast<size_t>(bh) * p.n_rows + gg) : gg;
-          if (static_cast<unsigned>(src) < static_cast<unsigned>(p.N))
-            vals[it] = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(bh) * p.N + src) * D + ch * 8));
-          else if (src != -1 && p.status != nullptr)
-            atomicCAS(p.status, 0, 1 /* ISA_ERR_INVALID_ARG: index out of range, row skipped */);
-        }
-      }
-#pragma unroll
-      for (int it = 0; it < CPR; ++it) {
-        const int c = it * 128 + r;
-        const int row = c / CPR, ch = c % CPR;
-        st_shared_v4(aQ + i * C::Q_BYTES + (ch >> 3) * (128 * 128) + sw128(row, ch & 7), vals[it].x, vals[it].y,
-                     vals[it].z, vals[it].w);
-      }
+      gather_rows_sw128<D>(p.q, p.row_idx, bh, p.n_rows, p.N, row0 + i * 128, r, aQ + i * C::Q_BYTES, true, p.status);
       fence_proxy_async_smem();
       mbar_arrive(&bars->q_full[i]);
     }
