@@ -71,9 +71,10 @@ def counts(cfg):
 FULL_TRAFFIC = {
     "config": "480p",
     # whole-wave launch (read + write), key-split launch (read + write), combine
-    "bytes": 398_867_456 + 40_851_456 + 14_972_672 + 8_448 + 18_467_840 + 0,
+    "bytes": 394_021_632 + 40_587_008 + 14_961_152 + 1_536 + 18_468_096 + 0,
     "sources": {
-        "sparse_attention_context_b200/csrc/flash2.cu": "fb5e1c53903090b2ec4ec14ea27383a3a30a47cbc8eb67d22a5b2b6505ba355c",
+        "sparse_attention_context_b200/csrc/flash2.cu": "a69fddf185ddeebee261af69fe5febba3d64c92f11b0083ef6b52262ff9f90aa",
+        "sparse_attention_context_b200/csrc/gather.cuh": "842e9958e7de511bd130413934b8da2dfcbd8ed14cef6f38ff09d728b527b34a",
         "sparse_attention_context_b200/csrc/tc_ptx.cuh": "1026ba5d3e08b740b9d4aa8f4fc7e2bd31b8c482744693570e460f8679e5be71",
     },
 }
