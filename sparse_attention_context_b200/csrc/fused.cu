@@ -177,10 +177,11 @@ __global__ void __launch_bounds__(352, 1)
     if (lane == 0) {
       bool ok = true;
       int g_issued = 0;
-      for (int g = 0; ok && g < total; ++g) {
-        const int k = g / nT, t = g % nT;
-        const int bh = item_of(k) / p.pairs_per_head;
-        const int r = bh * p.kv_rows_per_head + t * BN;
+      int t = 0, row_base = 0;  // key tile of g within its item, first K/V row of the item's head
+      for (int g = 0; ok && g < total; ++g, ++t) {
+        if (t == nT) t = 0;
+        if (t == 0) row_base = item_of(g / nT) / p.pairs_per_head * p.kv_rows_per_head;
+        const int r = row_base + t * BN;
 #pragma unroll
         for (int cc = 0; cc < C::NKC; ++cc) {
           if (g >= 1 && !(ok = fw1(&bars->k_empty[cc], (g - 1) & 1, bars, p))) break;
@@ -219,8 +220,9 @@ __global__ void __launch_bounds__(352, 1)
       // S_i(g) = Q_i (hi + lo) of key tile g, chunk by chunk of K: S_0 waits
       // for each chunk to land, S_1 (its last reader) releases each one;
       // commits s_full[i] (false: a wait gave up)
-      auto issue_S = [&](int i, int g) -> bool {
-        const int k = g / nT;
+      // (the issuing thread paces the tensor pipe: no divisions on its path;
+      // the item k and key tile t of g are carried along)
+      auto issue_S = [&](int i, int g, int k) -> bool {
         const uint32_t qa = aQ + ((k & 1) * 2 + i) * C::Q_BYTES;
         const uint32_t dS = tmem + i * BN;
 #pragma unroll
@@ -240,15 +242,12 @@ __global__ void __launch_bounds__(352, 1)
         umma_commit(&bars->s_full[i]);
         return true;
       };
-      // waits for the Q of key tile g's item (first tile of an item only)
-      auto q_ready = [&](int g) -> bool {
-        if (g % nT != 0) return true;
-        const int k = g / nT;
+      // waits for the Q of item k (before its first key tile)
+      auto q_ready = [&](int k) -> bool {
         return fw1(&bars->q_full[k & 1][0], (k >> 1) & 1, bars, p) &&
                fw1(&bars->q_full[k & 1][1], (k >> 1) & 1, bars, p);
       };
-      auto issue_PV = [&](int i, int g) -> bool {
-        const int k = g / nT, t = g % nT;
+      auto issue_PV = [&](int i, int g, int k, int t) -> bool {
         if (t == 0 && k > 0 && !fw1(&bars->o_free[i], (k - 1) & 1, bars, p)) return false;
         if (!fw1(&bars->p_full[i], g & 1, bars, p)) return false;
         tc_fence_after();
@@ -259,15 +258,23 @@ __global__ void __launch_bounds__(352, 1)
         umma_commit(&bars->o_done[i]);
         return true;
       };
-      if (total > 0) ok = q_ready(0) && issue_S(0, 0) && issue_S(1, 0);
+      if (total > 0) ok = q_ready(0) && issue_S(0, 0, 0) && issue_S(1, 0, 0);
+      int k = 0, t = 0;  // item and key tile of g
       for (int g = 0; ok && g < total; ++g) {
         const bool more = g + 1 < total;
+        int k1 = k, t1 = t + 1;  // of g + 1
+        if (t1 == nT) {
+          t1 = 0;
+          ++k1;
+        }
         if (!(ok = fw1(&bars->v_full, g & 1, bars, p))) break;
-        if (!(ok = issue_PV(0, g))) break;
-        if (more && !(ok = q_ready(g + 1) && issue_S(0, g + 1))) break;
-        if (!(ok = issue_PV(1, g))) break;
+        if (!(ok = issue_PV(0, g, k, t))) break;
+        if (more && !(ok = (t1 != 0 || q_ready(k1)) && issue_S(0, g + 1, k1))) break;
+        if (!(ok = issue_PV(1, g, k, t))) break;
         umma_commit(&bars->v_empty);
-        if (more && !(ok = issue_S(1, g + 1))) break;
+        if (more && !(ok = issue_S(1, g + 1, k1))) break;
+        k = k1;
+        t = t1;
       }
       umma_commit(&bars->teardown);
       mbar_wait_bounded(&bars->teardown, 0, nullptr, kWaitLimitNs);
