@@ -28,6 +28,12 @@ CASES = {
     "src_lt_block": CONFIGS["tiny"].replace(N_src=30, N_ctx=400, block=128, keep=0.5),
     "many_tiles": CONFIGS["tiny"].replace(H=1, d=128, N_src=3000, N_ctx=2900, block=128, keep=0.35, rho=0.25),
     "batch2": CONFIGS["tiny"].replace(B=2, H=3, d=128, N_src=700, N_ctx=450, block=128, keep=0.5, rho=0.2),
+    # block saliency over several 128-block tiles at d=64 (282 blocks: 3 row
+    # and column tiles, pad columns in the last)
+    "sal_tiles64": CONFIGS["tiny"].replace(H=2, d=64, N_src=9000, N_ctx=9000, block=64, keep=0.4, rho=0.1),
+    # the source segment ends exactly on a 128-block tile (nSB = 128): the
+    # context columns start a tile
+    "sal_edge128": CONFIGS["tiny"].replace(H=1, d=128, N_src=16384, N_ctx=10000, block=128, keep=0.3, rho=0.05),
 }
 
 
