@@ -813,7 +813,9 @@ def main():
                          f"scaled x{cfg.B * cfg.H / len(heads):g}"}
 
     nsm = torch.cuda.get_device_properties(dev).multi_processor_count
-    launches_per_step = 3 + 3 + full_stage_launches(cfg, n_keep, n_route, nsm)
+    # pre-selection: pooling, saliency, selection, and the value means of the
+    # kept context blocks; sharpness + Taylor: operand build, fused pass, route
+    launches_per_step = 3 + (1 if n_keep > 0 else 0) + 3 + full_stage_launches(cfg, n_keep, n_route, nsm)
     if rank == 0:
         rec = {"metric": METRIC, "value": round(ms_max, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": False,

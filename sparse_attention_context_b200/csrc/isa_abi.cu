@@ -194,6 +194,8 @@ int run_preselect(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint
   if (e == cudaSuccess)
     e = launch_select_ctx(at<float>(c.ws, c.L.partial), d.nChunks, at<float>(c.ws, c.L.sal), sal_user, kept, d.BH,
                           d.N_src, d.N_ctx, d.blk, d.n_keep, c.st);
+  if (e == cudaSuccess)
+    e = launch_pool_kept_v(v, kept, at<float>(c.ws, c.L.Vbar), d.BH, d.N_src, d.N_ctx, d.d, d.blk, d.n_keep, c.st);
   return cuda_status(e);
 }
 

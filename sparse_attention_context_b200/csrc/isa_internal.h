@@ -96,8 +96,8 @@ cudaError_t launch_fused(int D, const CUtensorMap& tmQ, const CUtensorMap& tmKhi
 cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                          const CUtensorMap& tmV, const FlashParams& p, int BH, cudaStream_t st);
 
-// Stage-1 kernels.  launch_pool writes fp32 Kbar and Vbar (Qbar too unless
-// it is null) and bf16 hi / lo of Qbar and Kbar
+// Stage-1 kernels.  launch_pool writes fp32 Kbar, Vbar of the source blocks
+// (Qbar too unless it is null) and bf16 hi / lo of Qbar and Kbar
 // into QKsplit: four [BH, nBp, D] arrays (Qhi, Qlo, Khi, Klo), nBp = nB
 // rounded up to 128, pad rows left unwritten.  launch_saliency_tc: partial
 // [BH, nBp/128, nCB] column sums per 128-row tile; launch_select_ctx adds
@@ -105,6 +105,10 @@ cudaError_t launch_attn2(int D, int BN, int mode, const CUtensorMap& tmQ, const 
 cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* Qbar, float* Kbar,
                         float* Vbar, uint16_t* QKsplit, int BH, int N_src, int N_ctx, int D, int blk,
                         cudaStream_t st);
+// Vbar rows of the kept context blocks (pool_kernel leaves the context rows
+// of Vbar unwritten), once kept [BH, n_keep] is known.
+cudaError_t launch_pool_kept_v(const uint16_t* v, const int32_t* kept, float* Vbar, int BH, int N_src, int N_ctx,
+                               int D, int blk, int n_keep, cudaStream_t st);
 cudaError_t launch_saliency_tc(const uint16_t* Qhi, const uint16_t* Qlo, const uint16_t* Khi, const uint16_t* Klo,
                                float* partial, int BH, int N_src, int N_ctx, int D, int blk, float scale,
                                int* status, cudaStream_t st);
