@@ -740,7 +740,7 @@ def main():
             api.isa_dense_attn_fwd(q, k, v, out=dout, ws=dws)
         d1.record(stream)
         torch.cuda.synchronize()
-        dense_ms = d0.elapsed_time(d1) / nd
+        dense_ms = max_over_ranks(d0.elapsed_time(d1) / nd, dev)
         assert api.isa_read_device_status(dws) == 0
         del dout
 
