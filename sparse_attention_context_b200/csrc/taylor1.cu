@@ -325,10 +325,12 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int ge = 0;  // ring elements issued: per key tile its Vbar tile, then its C_b
+      // ring elements issued: per key tile its Vbar tile, then its C_b
+      // (unsigned, so that % R and / R are bit operations)
+      unsigned ge = 0u;
       bool ok = true;
       int k_issued = 0;
-      auto slot_ready = [&](int e) -> bool {  // wait until ring slot e % R is free
+      auto slot_ready = [&](unsigned e) -> bool {  // wait until ring slot e % R is free
         return e < R || t1w(&bars->c_empty[e % R], ((e / R) - 1) & 1, bars, p);
       };
       for (int t = 0; ok && t < nT; ++t) {
@@ -341,7 +343,7 @@ __global__ void __launch_bounds__(320, 1)
         k_issued = t + 1;
         if (!(ok = slot_ready(ge))) break;
         {
-          const int r = ge % R;
+          const int r = static_cast<int>(ge % R);
           mbar_arrive_expect_tx(&bars->c_full[r], C::KT_BYTES);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(320, 1)
         const int nb = min(BN, nK - t * BN);
         for (int b = 0; b < nb; ++b) {
           if (!(ok = slot_ready(ge))) break;
-          const int r = ge % R;
+          const int r = static_cast<int>(ge % R);
           mbar_arrive_expect_tx(&bars->c_full[r], C::C_BYTES);
           const int crow = (bh * nK + t * BN + b) * D;
 #pragma unroll
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       // drain this thread's copies still in flight before the CTA may exit
       if (k_issued > 0) mbar_wait_bounded(&bars->k_full, (k_issued - 1) & 1, nullptr, kWaitLimitNs);
-      for (int e = ge > R ? ge - R : 0; e < ge; ++e)
+      for (unsigned e = ge > R ? ge - R : 0u; e < ge; ++e)
         mbar_wait_bounded(&bars->c_full[e % R], (e / R) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 9) {
@@ -371,7 +373,7 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t IDS = idesc_bf16(128, BN, 0);
       constexpr uint32_t IDO = idesc_bf16(128, D, 1);
       bool ok = t1w(&bars->q_full[0], 0, bars, p) && t1w(&bars->q_full[1], 0, bars, p);
-      int ge = 0;  // ring elements consumed (same order as the producer)
+      unsigned ge = 0u;  // ring elements consumed (same order as the producer; unsigned: bit-op % R)
       int na[2][2] = {{0, 0}, {0, 0}};
       for (int t = 0; ok && t < nT; ++t) {
         if (!(ok = t1w(&bars->k_full, t & 1, bars, p))) break;
@@ -384,7 +386,7 @@ __global__ void __launch_bounds__(320, 1)
           umma_commit(&bars->s_full[i]);
         }
         umma_commit(&bars->k_empty);
-        const int rv = ge % R;
+        const int rv = static_cast<int>(ge % R);
         if (!(ok = t1w(&bars->c_full[rv], (ge / R) & 1, bars, p))) break;
         const uint32_t aV = aC + rv * C::SLOT;
         for (int i = 0; i < 2 && ok; ++i) {
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(320, 1)
         ++ge;
         const int nb = min(BN, nK - t * BN);
         for (int b = 0; ok && b < nb; ++b, ++ge) {
-          const int r = ge % R, s = b & 1;
+          const int r = static_cast<int>(ge % R), s = b & 1;
           if (!(ok = t1w(&bars->c_full[r], (ge / R) & 1, bars, p))) break;
           const uint32_t cb = aC + r * C::SLOT;
           for (int i = 0; i < 2; ++i) {
