@@ -97,7 +97,11 @@ size_t isa_workspace_size(const isa_shape* shape);
  *                when n_keep == 0.
  *   saliency     [B, H, nCB] float out, or NULL.
  * The block means written into ws are inputs of isa_route_queries and
- * isa_attn_fwd; call this first with the same ws. */
+ * isa_attn_fwd; call this first with the same ws.  The means of v are
+ * pooled for the source blocks and for the context blocks this call keeps
+ * only (the others are never read), so the later calls on this ws must be
+ * given the kept set returned here: another one is reported as
+ * ISA_ERR_INVALID_ARG in the device status word (outputs undefined). */
 int isa_preselect_ctx(const isa_shape* shape, const uint16_t* q, const uint16_t* k,
                       const uint16_t* v, int32_t* kept_ctx_idx, float* saliency,
                       void* ws, size_t ws_bytes, void* stream);

@@ -23,7 +23,7 @@ struct Dims {
 };
 
 struct WsLayout {
-  size_t Kbar, Vbar, qksplit, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, rblk,
+  size_t Kbar, Vbar, ksel, qksplit, partial, sal, Khi, Klo, Vb, bias2, sharp, kept, routed, taylor, rblk,
       rrows, opart, mlpart, total;
   int split_ctas;  // key-split partial CTAs the workspace holds
 };
@@ -100,6 +100,7 @@ WsLayout layout(const Dims& d) {
   const size_t BH = d.BH;
   L.Kbar = take(BH * d.nB * d.d * 4);
   L.Vbar = take(BH * d.nB * d.d * 4);
+  L.ksel = take(BH * std::max(d.n_keep, 1) * 4);
   L.qksplit = take(4 * BH * d.nBp * d.d * 2);
   L.partial = take(BH * d.nChunks * std::max(d.nCB, 1) * 4);
   L.sal = take(BH * std::max(d.nCB, 1) * 4);
@@ -195,14 +196,15 @@ int run_preselect(const Ctx& c, const uint16_t* q, const uint16_t* k, const uint
     e = launch_select_ctx(at<float>(c.ws, c.L.partial), d.nChunks, at<float>(c.ws, c.L.sal), sal_user, kept, d.BH,
                           d.N_src, d.N_ctx, d.blk, d.n_keep, c.st);
   if (e == cudaSuccess)
-    e = launch_pool_kept_v(v, kept, at<float>(c.ws, c.L.Vbar), d.BH, d.N_src, d.N_ctx, d.d, d.blk, d.n_keep, c.st);
+    e = launch_pool_kept_v(v, kept, at<int32_t>(c.ws, c.L.ksel), at<float>(c.ws, c.L.Vbar), d.BH, d.N_src, d.N_ctx,
+                           d.d, d.blk, d.n_keep, c.st);
   return cuda_status(e);
 }
 
 int run_build_kept(const Ctx& c, const int32_t* kept) {
   const Dims& d = c.d;
   return cuda_status(launch_build_kept(at<float>(c.ws, c.L.Kbar), at<float>(c.ws, c.L.Vbar), kept,
-                                       at<uint16_t>(c.ws, c.L.Khi), at<uint16_t>(c.ws, c.L.Klo),
+                                       at<int32_t>(c.ws, c.L.ksel), at<uint16_t>(c.ws, c.L.Khi), at<uint16_t>(c.ws, c.L.Klo),
                                        at<uint16_t>(c.ws, c.L.Vb), at<float>(c.ws, c.L.bias2), d.BH, d.N_src,
                                        d.N_ctx, d.d, d.blk, d.n_keep, d.nKpad, c.status(), c.st));
 }

@@ -106,17 +106,18 @@ cudaError_t launch_pool(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         float* Vbar, uint16_t* QKsplit, int BH, int N_src, int N_ctx, int D, int blk,
                         cudaStream_t st);
 // Vbar rows of the kept context blocks (pool_kernel leaves the context rows
-// of Vbar unwritten), once kept [BH, n_keep] is known.
-cudaError_t launch_pool_kept_v(const uint16_t* v, const int32_t* kept, float* Vbar, int BH, int N_src, int N_ctx,
-                               int D, int blk, int n_keep, cudaStream_t st);
+// of Vbar unwritten), once kept [BH, n_keep] is known; the set is recorded
+// in ksel [BH, n_keep], which launch_build_kept checks its kept set against.
+cudaError_t launch_pool_kept_v(const uint16_t* v, const int32_t* kept, int32_t* ksel, float* Vbar, int BH,
+                               int N_src, int N_ctx, int D, int blk, int n_keep, cudaStream_t st);
 cudaError_t launch_saliency_tc(const uint16_t* Qhi, const uint16_t* Qlo, const uint16_t* Khi, const uint16_t* Klo,
                                float* partial, int BH, int N_src, int N_ctx, int D, int blk, float scale,
                                int* status, cudaStream_t st);
 cudaError_t launch_select_ctx(const float* partial, int n_chunks, float* sal_ws, float* sal_user, int32_t* kept,
                               int BH, int N_src, int N_ctx, int blk, int n_keep, cudaStream_t st);
-cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_t* kept, uint16_t* Khi,
-                              uint16_t* Klo, uint16_t* Vb, float* bias2, int BH, int N_src, int N_ctx, int D,
-                              int blk, int n_keep, int nKpad, int* status, cudaStream_t st);
+cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_t* kept, const int32_t* ksel,
+                              uint16_t* Khi, uint16_t* Klo, uint16_t* Vb, float* bias2, int BH, int N_src, int N_ctx,
+                              int D, int blk, int n_keep, int nKpad, int* status, cudaStream_t st);
 cudaError_t launch_route(const float* sharp, int32_t* routed, int32_t* taylor, int BH, int N, int n_route,
                          int* status, cudaStream_t st);
 // First-order Taylor variant (taylor1.cu).  cbuild: C_b = sum_j (k_j - Kbar_b)

@@ -106,16 +106,20 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
 
 // Vbar of the kept context blocks: one CTA per (kept slot, b*H + h), the
 // reduction of pool_kernel on v alone; slots with an index outside the
-// context are skipped (the operand build reports them).
+// context are skipped (the operand build reports them).  The kept set is
+// recorded in ksel, against which the operand build checks the set it is
+// given.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kept_v_kernel(const uint16_t* __restrict__ v,
-                                                          const int32_t* __restrict__ kept, float* __restrict__ Vbar,
-                                                          int N_src, int N_ctx, int blk, int nSB, int nB, int n_keep) {
+                                                          const int32_t* __restrict__ kept, int32_t* __restrict__ ksel,
+                                                          float* __restrict__ Vbar, int N_src, int N_ctx, int blk,
+                                                          int nSB, int nB, int n_keep) {
   constexpr int CPR = D / 8;
   constexpr int RG = 256 / CPR;
   __shared__ float red[RG][D + 4];
   const int slot = blockIdx.x, bh = blockIdx.y;
   const int c = __ldg(kept + static_cast<size_t>(bh) * n_keep + slot);
+  if (threadIdx.x == 0) ksel[static_cast<size_t>(bh) * n_keep + slot] = c;
   if (c < 0 || c >= nB - nSB) return;
   const int N = N_src + N_ctx;
   const int start = N_src + c * blk;
@@ -143,15 +147,15 @@ __global__ void __launch_bounds__(256) pool_kept_v_kernel(const uint16_t* __rest
   }
 }
 
-cudaError_t launch_pool_kept_v(const uint16_t* v, const int32_t* kept, float* Vbar, int BH, int N_src, int N_ctx,
-                               int D, int blk, int n_keep, cudaStream_t st) {
+cudaError_t launch_pool_kept_v(const uint16_t* v, const int32_t* kept, int32_t* ksel, float* Vbar, int BH,
+                               int N_src, int N_ctx, int D, int blk, int n_keep, cudaStream_t st) {
   const int nSB = (N_src + blk - 1) / blk, nCB = (N_ctx + blk - 1) / blk;
   if (n_keep <= 0 || nCB <= 0 || BH <= 0) return cudaSuccess;
   const dim3 grid(n_keep, BH);
   if (D == 128)
-    pool_kept_v_kernel<128><<<grid, 256, 0, st>>>(v, kept, Vbar, N_src, N_ctx, blk, nSB, nSB + nCB, n_keep);
+    pool_kept_v_kernel<128><<<grid, 256, 0, st>>>(v, kept, ksel, Vbar, N_src, N_ctx, blk, nSB, nSB + nCB, n_keep);
   else
-    pool_kept_v_kernel<64><<<grid, 256, 0, st>>>(v, kept, Vbar, N_src, N_ctx, blk, nSB, nSB + nCB, n_keep);
+    pool_kept_v_kernel<64><<<grid, 256, 0, st>>>(v, kept, ksel, Vbar, N_src, N_ctx, blk, nSB, nSB + nCB, n_keep);
   return cudaGetLastError();
 }
 

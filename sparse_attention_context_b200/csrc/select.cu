@@ -18,7 +18,10 @@
 //   writes the kept block numbers in ascending order.
 // build_kept_kernel: one CTA per kept block slot; writes the bf16 hi/lo split
 //   of Kbar, bf16 Vbar and log2(cnt) for the tensor-core stages; slots past
-//   the kept count are zero with a -inf bias.
+//   the kept count are zero with a -inf bias.  Vbar holds the context blocks
+//   that the pre-selection kept (ksel, its record of them), so a kept set
+//   that differs from it is reported (ISA_ERR_INVALID_ARG) rather than
+//   computed on block means that were never pooled.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -74,7 +77,8 @@ __global__ void __launch_bounds__(1024) select_ctx_kernel(const float* __restric
 
 template <int D>
 __global__ void build_kept_kernel(const float* __restrict__ Kbar, const float* __restrict__ Vbar,
-                                  const int32_t* __restrict__ kept, uint16_t* __restrict__ Khi,
+                                  const int32_t* __restrict__ kept, const int32_t* __restrict__ ksel,
+                                  uint16_t* __restrict__ Khi,
                                   uint16_t* __restrict__ Klo, uint16_t* __restrict__ Vb, float* __restrict__ bias2,
                                   int N_src, int N_ctx, int blk, int nSB, int nB, int n_keep, int nKpad,
                                   int* __restrict__ status) {
@@ -83,11 +87,14 @@ __global__ void build_kept_kernel(const float* __restrict__ Kbar, const float* _
   if (t < nSB) {
     b = t;
   } else if (t < nSB + n_keep) {
-    const int c = kept[static_cast<size_t>(bh) * n_keep + (t - nSB)];
+    const size_t ki = static_cast<size_t>(bh) * n_keep + (t - nSB);
+    const int c = kept[ki];
     if (c >= 0 && c < nB - nSB)
       b = nSB + c;
     else if (col == 0)
       atomicCAS(status, 0, 1 /* ISA_ERR_INVALID_ARG: kept block out of range, slot left empty */);
+    if (col == 0 && c != __ldg(ksel + ki))
+      atomicCAS(status, 0, 1 /* ISA_ERR_INVALID_ARG: not the pre-selection's kept set */);
   }
   const size_t dst = (static_cast<size_t>(bh) * nKpad + t) * D + col;
   if (b >= 0) {
@@ -117,17 +124,17 @@ cudaError_t launch_select_ctx(const float* partial, int n_chunks, float* sal_ws,
   return cudaGetLastError();
 }
 
-cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_t* kept, uint16_t* Khi,
-                              uint16_t* Klo, uint16_t* Vb, float* bias2, int BH, int N_src, int N_ctx, int D,
-                              int blk, int n_keep, int nKpad, int* status, cudaStream_t st) {
+cudaError_t launch_build_kept(const float* Kbar, const float* Vbar, const int32_t* kept, const int32_t* ksel,
+                              uint16_t* Khi, uint16_t* Klo, uint16_t* Vb, float* bias2, int BH, int N_src, int N_ctx,
+                              int D, int blk, int n_keep, int nKpad, int* status, cudaStream_t st) {
   const int nSB = (N_src + blk - 1) / blk, nCB = (N_ctx + blk - 1) / blk, nB = nSB + nCB;
   const dim3 grid(nKpad, BH);
   if (D == 128)
-    build_kept_kernel<128><<<grid, 128, 0, st>>>(Kbar, Vbar, kept, Khi, Klo, Vb, bias2, N_src, N_ctx, blk, nSB, nB,
-                                                 n_keep, nKpad, status);
+    build_kept_kernel<128><<<grid, 128, 0, st>>>(Kbar, Vbar, kept, ksel, Khi, Klo, Vb, bias2, N_src, N_ctx, blk, nSB,
+                                                 nB, n_keep, nKpad, status);
   else
-    build_kept_kernel<64><<<grid, 64, 0, st>>>(Kbar, Vbar, kept, Khi, Klo, Vb, bias2, N_src, N_ctx, blk, nSB, nB,
-                                               n_keep, nKpad, status);
+    build_kept_kernel<64><<<grid, 64, 0, st>>>(Kbar, Vbar, kept, ksel, Khi, Klo, Vb, bias2, N_src, N_ctx, blk, nSB,
+                                               nB, n_keep, nKpad, status);
   return cudaGetLastError();
 }
 

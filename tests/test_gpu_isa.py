@@ -133,3 +133,29 @@ def _sets(q, k, v, cfg):
     the host path computes too)."""
     g = run_fused(cfg, q, k, v)
     return {key: g[key] for key in ("kept", "sal", "sharp", "routed", "taylor")}
+
+
+def test_other_kept_set_is_reported(cuda_ok):
+    """The mean of v over a context block is pooled only when the
+    pre-selection keeps that block: a later stage given another (valid)
+    kept set reports ISA_ERR_INVALID_ARG in the device status word instead
+    of computing on means that were never pooled."""
+    cfg = CASES["many_tiles"]
+    _, (q, k, v) = inputs(cfg)
+    shape = api.make_shape(q, cfg.N_src, cfg.block, cfg.keep, cfg.rho)
+    ws = api.new_workspace(shape)
+    kept, _ = api.isa_preselect_ctx(q, k, v, shape, ws)
+    torch.cuda.synchronize()
+    assert api.isa_read_device_status(ws) == 0
+    api.isa_route_queries(q, kept, shape, ws)  # the same set: fine
+    torch.cuda.synchronize()
+    assert api.isa_read_device_status(ws) == 0
+    nCB = -(-cfg.N_ctx // cfg.block)
+    chosen = kept[0, 0].cpu().tolist()
+    unused = next(c for c in range(nCB) if c not in chosen)
+    other = kept.clone()
+    other[0, 0] = torch.tensor(sorted(chosen[1:] + [unused]), dtype=kept.dtype, device=kept.device)
+    api.isa_route_queries(q, other, shape, ws)
+    torch.cuda.synchronize()
+    assert api.isa_read_device_status(ws) == 1  # ISA_ERR_INVALID_ARG
+
