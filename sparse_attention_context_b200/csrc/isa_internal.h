@@ -12,7 +12,7 @@ namespace isa {
 constexpr int kStatusOffset = 0;   // int32 in the workspace control block
 constexpr int kInjectOffset = 4;   // int32 fault-injection word (tests)
 constexpr int kCtlBytes = 256;
-constexpr int kTopkCap = 4096;     // max context blocks the top-k sort holds
+constexpr int kTopkCap = 4096;     // max context blocks per head the selection kernel holds
 constexpr int kRouteBlocksCap = 16384;  // max query blocks per head of the block grouping
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
